@@ -1,0 +1,301 @@
+"""Python binding of libbsa.so: dynamic block-sparse attention on B200 (sm_100a).
+
+Thin ctypes marshalling over the C ABI in include/bsa.h. Every step of the method
+runs in the library's CUDA kernels; torch only owns device memory and streams.
+Importing this package does not load the library; the first call does, and it
+raises if libbsa.so is missing (build it with ``python -m
+block_sparse_long_06_b200.build``). There is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsa.so")
+
+BSA_OK, BSA_ERR_INVALID_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_WORKSPACE, BSA_ERR_CUDA = range(5)
+BSA_DEV_BAD_PAGE, BSA_DEV_BAD_KEPT, BSA_DEV_NONFINITE, BSA_DEV_TIMEOUT, BSA_DEV_FP16_RANGE = (
+    0x1, 0x2, 0x4, 0x8, 0x10)
+PHASE_DECODE, PHASE_PREFILL = 0, 1
+OP_SCORE, OP_SELECT, OP_DECODE, OP_PREFILL = 0, 1, 2, 3
+BLOCK = 64
+
+EXPORTED = ["bsa_max_kept", "bsa_workspace_size", "bsa_score_blocks", "bsa_select_top_p",
+            "bsa_decode", "bsa_prefill", "bsa_status_string", "bsa_last_cuda_error"]
+
+
+class BsaError(RuntimeError):
+    pass
+
+
+class CCache(ctypes.Structure):
+    _fields_ = [("base", ctypes.c_void_p), ("seq_stride", ctypes.c_int64),
+                ("block_stride", ctypes.c_int64), ("head_stride", ctypes.c_int64),
+                ("page_table", ctypes.c_void_p), ("page_table_stride", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("extent", ctypes.c_int64)]
+
+
+class CProblem(ctypes.Structure):
+    _fields_ = [("phase", ctypes.c_int32), ("B", ctypes.c_int32), ("Hq", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("r", ctypes.c_int32),
+                ("block", ctypes.c_int32), ("T", ctypes.c_int32), ("seq_lens", ctypes.c_void_p),
+                ("n_sink", ctypes.c_int32), ("n_local", ctypes.c_int32),
+                ("k_max", ctypes.c_int32), ("k_min", ctypes.c_int32), ("p", ctypes.c_float),
+                ("idx_scale", ctypes.c_float), ("attn_scale", ctypes.c_float),
+                ("head_w", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libbsa.so once and declare its signatures; raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise BsaError(f"{path} not found: build it with `python -m block_sparse_long_06_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(CProblem)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    lib.bsa_max_kept.argtypes = [P]
+    lib.bsa_max_kept.restype = ctypes.c_int32
+    lib.bsa_workspace_size.argtypes = [P, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.bsa_workspace_size.restype = ctypes.c_int
+    lib.bsa_score_blocks.argtypes = [P, vp, CCache, vp, vp, vp]
+    lib.bsa_score_blocks.restype = ctypes.c_int
+    lib.bsa_select_top_p.argtypes = [P, vp, vp, vp, vp, vp]
+    lib.bsa_select_top_p.restype = ctypes.c_int
+    for name in ("bsa_decode", "bsa_prefill"):
+        f = getattr(lib, name)
+        f.argtypes = [P, vp, CCache, CCache, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+        f.restype = ctypes.c_int
+    lib.bsa_status_string.argtypes = [ctypes.c_int]
+    lib.bsa_status_string.restype = ctypes.c_char_p
+    lib.bsa_last_cuda_error.argtypes = []
+    lib.bsa_last_cuda_error.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str):
+    if status != BSA_OK:
+        lib = load_library()
+        msg = lib.bsa_status_string(status).decode()
+        if status == BSA_ERR_CUDA:
+            msg += ": " + lib.bsa_last_cuda_error().decode()
+        raise BsaError(f"{what}: {msg} (status {status})")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ------------------------------------------------------------------ problem / caches
+@dataclass
+class Problem:
+    phase: int
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    T: int
+    n_sink: int
+    n_local: int
+    k_max: int
+    p: float
+    k_min: int = 0
+    r: int = 16
+    block: int = BLOCK
+    idx_scale: float = 0.0        # 0 -> 1/sqrt(r)
+    attn_scale: float = 0.0       # 0 -> 1/sqrt(d)
+    seq_lens: Optional[torch.Tensor] = None   # device int32 [B] (decode)
+    head_w: Optional[torch.Tensor] = None     # device float32 [Hq]
+
+    @property
+    def G(self):
+        return self.Hq // self.Hkv
+
+    @property
+    def nb(self):
+        return (self.T + BLOCK - 1) // BLOCK
+
+    def c(self) -> CProblem:
+        return CProblem(self.phase, self.B, self.Hq, self.Hkv, self.d, self.r, self.block, self.T,
+                        _ptr(self.seq_lens), self.n_sink, self.n_local, self.k_max, self.k_min,
+                        float(self.p), float(self.idx_scale), float(self.attn_scale),
+                        _ptr(self.head_w))
+
+
+@dataclass
+class Cache:
+    """A bf16 cache tensor (K, V or index keys) and its addressing (bsa_cache_t)."""
+    tensor: torch.Tensor
+    seq_stride: int
+    block_stride: int
+    head_stride: int
+    page_table: Optional[torch.Tensor] = None
+    num_pages: int = 0
+
+    def c(self) -> CCache:
+        pt = self.page_table
+        return CCache(self.tensor.data_ptr(), self.seq_stride, self.block_stride, self.head_stride,
+                      None if pt is None else pt.data_ptr(),
+                      0 if pt is None else pt.shape[1], self.num_pages, self.tensor.numel())
+
+
+def contiguous_cache(t: torch.Tensor) -> Cache:
+    """[B, Hkv, T, w] contiguous bf16 tensor."""
+    assert t.is_contiguous() and t.dtype == torch.bfloat16 and t.dim() == 4
+    B, H, T, w = t.shape
+    return Cache(t, H * T * w, BLOCK * w, T * w)
+
+
+def paged_cache(pool: torch.Tensor, page_table: torch.Tensor) -> Cache:
+    """[P, Hkv, 64, w] contiguous bf16 pool with a [B, nb] int32 page table."""
+    assert pool.is_contiguous() and pool.dtype == torch.bfloat16 and pool.shape[2] == BLOCK
+    assert page_table.dtype == torch.int32 and page_table.is_contiguous()
+    P, H, _, w = pool.shape
+    return Cache(pool, 0, H * BLOCK * w, BLOCK * w, page_table, P)
+
+
+# ------------------------------------------------------------------ the C entry points
+def bsa_max_kept(prob: Problem) -> int:
+    return load_library().bsa_max_kept(ctypes.byref(prob.c()))
+
+
+def bsa_workspace_size(prob: Problem, op: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load_library().bsa_workspace_size(ctypes.byref(prob.c()), op, ctypes.byref(out)),
+           "bsa_workspace_size")
+    return out.value
+
+
+def bsa_score_blocks(prob: Problem, q_idx, k_idx: Cache, block_scores, dev_status=None,
+                     stream=None):
+    _check(load_library().bsa_score_blocks(ctypes.byref(prob.c()), _ptr(q_idx), k_idx.c(),
+                                           _ptr(block_scores), _ptr(dev_status), _stream(stream)),
+           "bsa_score_blocks")
+
+
+def bsa_select_top_p(prob: Problem, block_scores, kept, kept_count, dev_status=None, stream=None):
+    _check(load_library().bsa_select_top_p(ctypes.byref(prob.c()), _ptr(block_scores), _ptr(kept),
+                                           _ptr(kept_count), _ptr(dev_status), _stream(stream)),
+           "bsa_select_top_p")
+
+
+def bsa_decode(prob: Problem, q, k: Cache, v: Cache, kept, kept_count, o, lse, o_f32, workspace,
+               dev_status=None, stream=None):
+    _check(load_library().bsa_decode(ctypes.byref(prob.c()), _ptr(q), k.c(), v.c(), _ptr(kept),
+                                     _ptr(kept_count), _ptr(o), _ptr(lse), _ptr(o_f32),
+                                     _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                     _ptr(dev_status), _stream(stream)),
+           "bsa_decode")
+
+
+def bsa_prefill(prob: Problem, q, k: Cache, v: Cache, kept, kept_count, o, lse, o_f32, workspace,
+                dev_status=None, stream=None):
+    _check(load_library().bsa_prefill(ctypes.byref(prob.c()), _ptr(q), k.c(), v.c(), _ptr(kept),
+                                      _ptr(kept_count), _ptr(o), _ptr(lse), _ptr(o_f32),
+                                      _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                      _ptr(dev_status), _stream(stream)),
+           "bsa_prefill")
+
+
+def bsa_status_string(status: int) -> str:
+    return load_library().bsa_status_string(status).decode()
+
+
+# ------------------------------------------------------------------ pipelines
+class DecodeStep:
+    """Buffers for one decode problem and the score -> select -> attend chain.
+
+    Outputs live in this object (torch-allocated once); ``run`` enqueues the three
+    entry points on the current stream and returns nothing (no host sync)."""
+
+    def __init__(self, prob: Problem, device="cuda", keep_f32=True):
+        assert prob.phase == PHASE_DECODE
+        self.prob = prob
+        dev = torch.device(device)
+        mk = bsa_max_kept(prob)
+        self.scores = torch.empty(prob.B, prob.Hkv, prob.nb, dtype=torch.float32, device=dev)
+        self.kept = torch.empty(prob.B, prob.Hkv, mk, dtype=torch.int32, device=dev)
+        self.kept_count = torch.empty(prob.B, prob.Hkv, dtype=torch.int32, device=dev)
+        self.o = torch.empty(prob.B, prob.Hq, prob.d, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(prob.B, prob.Hq, dtype=torch.float32, device=dev)
+        self.o_f32 = (torch.empty(prob.B, prob.Hq, prob.d, dtype=torch.float32, device=dev)
+                      if keep_f32 else None)
+        ws = bsa_workspace_size(prob, OP_DECODE)
+        self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def run(self, q, q_idx, k_idx: Cache, k: Cache, v: Cache, stream=None):
+        p = self.prob
+        bsa_score_blocks(p, q_idx, k_idx, self.scores, self.status, stream)
+        bsa_select_top_p(p, self.scores, self.kept, self.kept_count, self.status, stream)
+        bsa_decode(p, q, k, v, self.kept, self.kept_count, self.o, self.lse, self.o_f32,
+                   self.workspace, self.status, stream)
+
+
+class Prefill:
+    """Buffers for one prefill problem and the score -> select -> attend chain."""
+
+    def __init__(self, prob: Problem, device="cuda", keep_f32=True):
+        assert prob.phase == PHASE_PREFILL
+        self.prob = prob
+        dev = torch.device(device)
+        nqb = prob.nb
+        mk = bsa_max_kept(prob)
+        self.scores = torch.empty(prob.B, prob.Hkv, nqb, nqb, dtype=torch.float32, device=dev)
+        self.kept = torch.empty(prob.B, prob.Hkv, nqb, mk, dtype=torch.int32, device=dev)
+        self.kept_count = torch.empty(prob.B, prob.Hkv, nqb, dtype=torch.int32, device=dev)
+        self.o = torch.empty(prob.B, prob.Hq, prob.T, prob.d, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(prob.B, prob.Hq, prob.T, dtype=torch.float32, device=dev)
+        self.o_f32 = (torch.empty(prob.B, prob.Hq, prob.T, prob.d, dtype=torch.float32, device=dev)
+                      if keep_f32 else None)
+        ws = bsa_workspace_size(prob, OP_PREFILL)
+        self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def select(self, q_idx, k_idx: Cache, stream=None):
+        bsa_score_blocks(self.prob, q_idx, k_idx, self.scores, self.status, stream)
+        bsa_select_top_p(self.prob, self.scores, self.kept, self.kept_count, self.status, stream)
+
+    def attend(self, q, k: Cache, v: Cache, stream=None):
+        bsa_prefill(self.prob, q, k, v, self.kept, self.kept_count, self.o, self.lse, self.o_f32,
+                    self.workspace, self.status, stream)
+
+    def run(self, q, q_idx, k_idx: Cache, k: Cache, v: Cache, stream=None):
+        self.select(q_idx, k_idx, stream)
+        self.attend(q, k, v, stream)
+
+
+def problem_for(w, seq_lens: Optional[torch.Tensor] = None,
+                head_w: Optional[torch.Tensor] = None) -> Problem:
+    """Problem description of a synthetic workload (see workloads.Workload)."""
+    phase = PHASE_DECODE if w.phase == "decode" else PHASE_PREFILL
+    return Problem(phase=phase, B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, n_sink=w.n_sink,
+                   n_local=w.n_local, k_max=w.k_max, k_min=w.k_min, p=w.p, r=w.r,
+                   idx_scale=1.0 / math.sqrt(w.r), attn_scale=1.0 / math.sqrt(w.d),
+                   seq_lens=seq_lens if phase == PHASE_DECODE else None, head_w=head_w)
+
+
+def caches_for(inputs: dict):
+    """(k_idx, K, V) caches of a generated input dict."""
+    k_idx = contiguous_cache(inputs["k_idx"])
+    if inputs.get("page_table") is not None:
+        pt = inputs["page_table"]
+        return k_idx, paged_cache(inputs["K"], pt), paged_cache(inputs["V"], pt)
+    return k_idx, contiguous_cache(inputs["K"]), contiguous_cache(inputs["V"])

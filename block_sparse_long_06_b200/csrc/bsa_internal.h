@@ -1,0 +1,97 @@
+// Internal launch interface between the C ABI (bsa_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/bsa.h"
+
+namespace bsa {
+
+// Device-side copy of a bsa_cache_t (strides in elements).
+struct CacheView {
+  const void* base;
+  int64_t seq_stride, block_stride, head_stride;
+  const int32_t* page_table;
+  int32_t pt_stride, num_pages;
+  int64_t extent;
+};
+
+struct ScoreDecodeArgs {
+  const void* q_idx;          // [B, Hq, 16] bf16
+  CacheView kidx;             // width 16
+  const int32_t* seq_lens;    // [B] or null
+  const float* head_w;        // [Hq] or null
+  float* scores;              // [B*Hkv, nb_max]
+  int32_t* status;
+  int B, Hq, Hkv, G, T, nb_max, chunks_per_row;
+  int64_t total_items;
+  float idx_scale;
+};
+
+struct ScorePrefillArgs {
+  const void* q_idx;          // [B, Hq, T, 16] bf16
+  CacheView kidx;             // width 16
+  const float* head_w;
+  float* scores;              // [B*Hkv, nqb, nqb]
+  int32_t* status;
+  int B, Hq, Hkv, G, T, nqb;
+  float idx_scale;
+};
+
+struct SelectArgs {
+  const float* scores;
+  int32_t* kept;
+  int32_t* kept_count;
+  const int32_t* seq_lens;
+  int32_t* status;
+  int phase, B, Hkv, T, nb_max, nqb, max_kept;
+  int n_sink, n_local, k_max, k_min;
+  float p;
+};
+
+struct DecodeArgs {
+  const void* q;              // [B, Hq, d] bf16
+  CacheView k, v;
+  const int32_t* kept;        // [B*Hkv, max_kept]
+  const int32_t* kept_count;  // [B*Hkv]
+  const int32_t* seq_lens;
+  void* o;                    // [B, Hq, d] bf16
+  float* lse;                 // [B, Hq]
+  float* o_f32;               // [B, Hq, d] or null
+  float* part_o;              // [units, G, d]
+  float* part_ml;             // [units, G, 2]
+  int32_t* status;
+  int B, Hq, Hkv, G, d, T, max_kept, splits, split_len;
+  float scale_log2;           // attn_scale * log2(e)
+};
+
+struct PrefillArgs {
+  const void* q;              // [B, Hq, T, d] bf16
+  CacheView k, v;
+  const void* v16;            // [B*Hkv, Tpad, d] fp16 (workspace copy of V)
+  const int32_t* kept;        // [B*Hkv*nqb, max_kept]
+  const int32_t* kept_count;  // [B*Hkv*nqb]
+  void* o;                    // [B, Hq, T, d] bf16
+  float* lse;                 // [B, Hq, T]
+  float* o_f32;               // or null
+  int32_t* status;
+  int B, Hq, Hkv, G, d, T, nqb, Tpad, max_kept;
+  float scale_log2;
+};
+
+// Each launcher returns the cudaError_t of its launch.
+cudaError_t launch_score_decode(const ScoreDecodeArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_score_prefill(const ScorePrefillArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                          int num_units, int num_sms, cudaStream_t s);
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                           const CUtensorMap& tv16, int num_sms, cudaStream_t s);
+cudaError_t launch_v_to_f16(const PrefillArgs& a, cudaStream_t s);
+
+// Decode split-K geometry chosen on the host from the worst-case kept count.
+void decode_split_plan(int rows, int max_kept, int num_sms, int* splits, int* split_len);
+
+}  // namespace bsa

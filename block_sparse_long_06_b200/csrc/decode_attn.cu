@@ -1,0 +1,432 @@
+// Split-K sparse flash-decode over the kept blocks, then an LSE merge.
+//
+// For each query head h of kv group g of sequence b: exact softmax attention over
+// the tokens t < T_b of the kept 64-token blocks (HGA, Central mechanism §4 and
+// Key contributions §2: exact token-level attention over the routed set).
+//
+// Design (HBM-bound: 2 * 64 * d * 2 bytes of K/V per kept block per (b, g)):
+//  * work unit = (row (b, g), split s) = a slice of split_len consecutive entries
+//    of the row's kept list; persistent CTAs (one per SM) stride over the units;
+//  * one producer warp streams each kept block's K and V tiles into a ring of
+//    shared-memory stages with TMA (2-D tensor maps, 128-byte swizzle, one box =
+//    64 tokens x 64 dims), completion on per-stage "full" mbarriers; four
+//    consumer warps release stages through "empty" mbarriers;
+//  * consumer warp w owns tokens [16w, 16w+16) of every block: S^T = K_w Q^T on
+//    mma.m16n8k16 (tokens as M, the group's heads as N), online softmax in fp32
+//    (log2 domain), then O^T += V_w^T P^T (V^T via ldmatrix.trans, P^T moved into
+//    the B-fragment layout with movmatrix). P is split into bf16 hi + lo parts, so
+//    the P.V products keep ~16 mantissa bits;
+//  * at the end of a unit the four warps' (m, l, O) are merged in shared memory
+//    and written as one partial; the merge kernel combines the splits of a row
+//    with their log-sum-exp weights and writes o (bf16), o_f32 and lse.
+#include "bsa_common.cuh"
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+
+template <int D>
+struct DecodeCfg {
+  static constexpr int kBoxes = D / 64;                       // 64-dim boxes per tile
+  static constexpr int kTileBytes = kBlock * D * 2;           // one K or V tile
+  static constexpr int kStageBytes = 2 * kTileBytes;          // K + V
+  static constexpr int kStages = D == 128 ? 5 : 8;
+  static constexpr int kKsteps = D / 16;
+};
+
+template <int D, int NT>
+struct DecodeSmem {
+  static constexpr int kRing = DecodeCfg<D>::kStages * DecodeCfg<D>::kStageBytes;
+  static constexpr int kComb = kConsumerWarps * (NT * 8) * D * 4;   // partial O per warp
+  static constexpr int kStats = kConsumerWarps * (NT * 8) * 2 * 4;  // m, l per warp
+  static constexpr int kBars = 2 * DecodeCfg<D>::kStages * 8;
+  static constexpr int kInfo = DecodeCfg<D>::kStages * 4;
+  static constexpr int kTotal = kRing + kComb + kStats + kBars + kInfo + 1024;  // + alignment
+};
+
+BSA_DEVFN void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32)); }
+// Barrier over the consumer warps that also ANDs a flag across them, so a
+// decision to stop is taken by all of them together.
+BSA_DEVFN bool consumer_sync_and(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n bar.red.and.pred po, 1, %2, pi;\n"
+      " selp.u32 %0, 1, 0, po;\n}\n"
+      : "=r"(out)
+      : "r"(static_cast<uint32_t>(v)), "n"(kConsumerWarps * 32));
+  return out != 0;
+}
+
+BSA_DEVFN int seq_len(const DecodeArgs& a, int b) {
+  int Tb = a.seq_lens ? a.seq_lens[b] : a.T;
+  return Tb < 0 ? 0 : (Tb > a.T ? a.T : Tb);
+}
+
+// Row (in rows of width d) of the first token of block `blk` of (b, g); -1 if invalid.
+BSA_DEVFN int64_t tile_row(const CacheView& c, int b, int g, int blk, int d) {
+  int64_t phys = blk;
+  if (c.page_table != nullptr) {
+    phys = c.page_table[static_cast<int64_t>(b) * c.pt_stride + blk];
+    if (phys < 0 || phys >= c.num_pages) return -1;
+  }
+  const int64_t off = static_cast<int64_t>(b) * c.seq_stride + phys * c.block_stride +
+                      static_cast<int64_t>(g) * c.head_stride;
+  if (off < 0 || off + static_cast<int64_t>(kBlock) * d > c.extent) return -1;
+  return off / d;
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_attn_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
+                       const __grid_constant__ CUtensorMap tmv, const int num_units) {
+  using Cfg = DecodeCfg<D>;
+  using Sm = DecodeSmem<D, NT>;
+  constexpr int S = Cfg::kStages;
+  constexpr int NH = NT * 8;  // padded heads
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* ring = smem;
+  float* comb = reinterpret_cast<float*>(smem + Sm::kRing);
+  float* stats = reinterpret_cast<float*>(smem + Sm::kRing + Sm::kComb);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Sm::kRing + Sm::kComb + Sm::kStats);
+  uint64_t* empty = full + S;
+  int* sinfo = reinterpret_cast<int*>(empty + S);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmk);
+      prefetch_tensormap(&tmv);
+      uint32_t it = 0;
+      bool ok_all = true;
+      for (int unit = blockIdx.x; unit < num_units && ok_all; unit += gridDim.x) {
+        const int row = unit / a.splits, sp = unit % a.splits;
+        const int b = row / a.Hkv, g = row % a.Hkv;
+        const int cnt = min(a.kept_count[row], a.max_kept);
+        const int e0 = sp * a.split_len, e1 = min(cnt, e0 + a.split_len);
+        const int nb = (seq_len(a, b) + kBlock - 1) / kBlock;
+        for (int e = e0; e < e1; ++e, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
+            report(a.status, BSA_DEV_TIMEOUT);
+            ok_all = false;
+            break;
+          }
+          const int blk = a.kept[static_cast<int64_t>(row) * a.max_kept + e];
+          int64_t rk = -1, rv = -1;
+          if (blk >= 0 && blk < nb) {
+            rk = tile_row(a.k, b, g, blk, D);
+            rv = tile_row(a.v, b, g, blk, D);
+            if (rk < 0 || rv < 0) report(a.status, BSA_DEV_BAD_PAGE);
+          } else {
+            report(a.status, BSA_DEV_BAD_KEPT);
+          }
+          const bool ok = rk >= 0 && rv >= 0;
+          sinfo[s] = ok ? blk : -1;
+          unsigned char* st = ring + s * Cfg::kStageBytes;
+          if (ok) {
+            mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
+#pragma unroll
+            for (int x = 0; x < Cfg::kBoxes; ++x) {
+              tma_load_2d(st + x * 8192, &tmk, x * 64, static_cast<int32_t>(rk), &full[s]);
+              tma_load_2d(st + Cfg::kTileBytes + x * 8192, &tmv, x * 64, static_cast<int32_t>(rv),
+                          &full[s]);
+            }
+          } else {
+            mbar_arrive(&full[s]);
+          }
+        }
+      }
+      // drain: wait until the consumers released every stage we filled (bounded)
+      for (uint32_t k = 0; k < S && k < it; ++k) {
+        const uint32_t j = it - 1 - k;
+        mbar_wait(&empty[j % S], (j / S) & 1, 200000000ull);
+      }
+    }
+    return;
+  }
+
+  // --------------------------------------------------------------- consumers
+  const int gid = lane >> 2, tig = lane & 3;
+  const int rr = lane & 7, mi = lane >> 3;
+  uint32_t it = 0;
+  bool alive = true;
+  for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x) {
+    const int row = unit / a.splits, sp = unit % a.splits;
+    const int b = row / a.Hkv, g = row % a.Hkv;
+    const int cnt = min(a.kept_count[row], a.max_kept);
+    const int e0 = sp * a.split_len, e1 = min(cnt, e0 + a.split_len);
+    const int Tb = seq_len(a, b);
+
+    // Q^T fragments: head (8*nt + gid) of the group, dims 16ks + 2tig (+1), +8
+    uint32_t bq[NT][Cfg::kKsteps][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int hl = nt * 8 + gid;
+      const bool hv = hl < a.G;
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+          static_cast<const char*>(a.q) +
+          ((static_cast<int64_t>(b) * a.Hq + g * a.G + (hv ? hl : 0)) * D) * 2);
+#pragma unroll
+      for (int ks = 0; ks < Cfg::kKsteps; ++ks) {
+        bq[nt][ks][0] = hv ? qrow[(ks * 16 + 2 * tig) / 2] : 0u;
+        bq[nt][ks][1] = hv ? qrow[(ks * 16 + 8 + 2 * tig) / 2] : 0u;
+      }
+    }
+    float m[NT][2], l[NT][2];
+    float acc[NT][Cfg::kKsteps][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m[nt][0] = m[nt][1] = -INFINITY;
+      l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < Cfg::kKsteps; ++mt)
+        acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
+    }
+
+    for (int e = e0; e < e1 && alive; ++e, ++it) {
+      const int s = it % S;
+      if (!mbar_wait(&full[s], (it / S) & 1)) {
+        if (lane == 0) report(a.status, BSA_DEV_TIMEOUT);
+        alive = false;
+        break;
+      }
+      const int blk = sinfo[s];
+      if (blk >= 0) {
+        const uint32_t kb = smem_u32(ring + s * Cfg::kStageBytes);
+        const uint32_t vb = kb + Cfg::kTileBytes;
+        const int valid = Tb - blk * kBlock - 16 * warp;  // tokens of this warp that exist
+        // ---- S^T = K_w Q^T
+        float sc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < Cfg::kKsteps; ++ks) {
+          const int trow = 16 * warp + rr + 8 * (mi & 1);
+          const int chunk = 2 * ks + (mi >> 1);
+          uint32_t af[4];
+          ldsm_x4(af, kb + (chunk >> 3) * 8192 + swz128(trow, chunk & 7));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_bf16(sc[nt], af, bq[nt][ks][0], bq[nt][ks][1]);
+        }
+        // ---- online softmax (log2 domain) per head column
+        const bool v0 = gid < valid, v1 = gid + 8 < valid;
+        uint32_t phi[NT][2], plo[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float p[4];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const float s0 = v0 ? sc[nt][c] * a.scale_log2 : -INFINITY;
+            const float s1 = v1 ? sc[nt][2 + c] * a.scale_log2 : -INFINITY;
+            float mx = fmaxf(s0, s1);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float mnew = fmaxf(m[nt][c], mx);
+            const float base = mnew == -INFINITY ? 0.f : mnew;
+            const float corr = ex2(m[nt][c] - base);
+            m[nt][c] = mnew;
+            p[c] = ex2(s0 - base);
+            p[2 + c] = ex2(s1 - base);
+            l[nt][c] = l[nt][c] * corr + p[c] + p[2 + c];
+#pragma unroll
+            for (int mt = 0; mt < Cfg::kKsteps; ++mt) {
+              acc[nt][mt][c] *= corr;
+              acc[nt][mt][2 + c] *= corr;
+            }
+          }
+          // P^T B-fragments (hi and lo bf16 parts)
+          const uint32_t h0 = pack_bf16(p[0], p[1]);
+          const uint32_t h1 = pack_bf16(p[2], p[3]);
+          const float2 f0 = unpack_bf16(h0), f1 = unpack_bf16(h1);
+          const uint32_t l0 = pack_bf16(p[0] - f0.x, p[1] - f0.y);
+          const uint32_t l1 = pack_bf16(p[2] - f1.x, p[3] - f1.y);
+          phi[nt][0] = movmatrix_t(h0);
+          phi[nt][1] = movmatrix_t(h1);
+          plo[nt][0] = movmatrix_t(l0);
+          plo[nt][1] = movmatrix_t(l1);
+        }
+        // ---- O^T += V_w^T P^T
+        const bool partial = valid < 16;
+#pragma unroll
+        for (int mt = 0; mt < Cfg::kKsteps; ++mt) {
+          const int trow = 16 * warp + rr + 8 * (mi >> 1);
+          const int chunk = 2 * mt + (mi & 1);
+          uint32_t af[4];
+          ldsm_x4_t(af, vb + (chunk >> 3) * 8192 + swz128(trow, chunk & 7));
+          if (partial) {
+            // zero V of tokens that do not exist (their P is 0; avoid 0 * NaN)
+            const int t0 = 2 * tig, t1 = 2 * tig + 8;
+            const uint32_t m0 = (t0 < valid ? 0x0000ffffu : 0u) | (t0 + 1 < valid ? 0xffff0000u : 0u);
+            const uint32_t m1 = (t1 < valid ? 0x0000ffffu : 0u) | (t1 + 1 < valid ? 0xffff0000u : 0u);
+            af[0] &= m0;
+            af[1] &= m0;
+            af[2] &= m1;
+            af[3] &= m1;
+          }
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_bf16(acc[nt][mt], af, phi[nt][0], phi[nt][1]);
+            mma_bf16(acc[nt][mt], af, plo[nt][0], plo[nt][1]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+
+    // ---- merge the four warps' partials of this unit
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float lv = l[nt][c];
+        lv += __shfl_xor_sync(0xffffffffu, lv, 4);
+        lv += __shfl_xor_sync(0xffffffffu, lv, 8);
+        lv += __shfl_xor_sync(0xffffffffu, lv, 16);
+        const int h = nt * 8 + 2 * tig + c;
+        if (gid == 0) {
+          stats[(warp * NH + h) * 2 + 0] = m[nt][c];
+          stats[(warp * NH + h) * 2 + 1] = lv;
+        }
+#pragma unroll
+        for (int mt = 0; mt < Cfg::kKsteps; ++mt) {
+          comb[(warp * NH + h) * D + 16 * mt + gid] = acc[nt][mt][c];
+          comb[(warp * NH + h) * D + 16 * mt + gid + 8] = acc[nt][mt][2 + c];
+        }
+      }
+    }
+    consumer_sync();
+    const int tid = threadIdx.x;
+    for (int x = tid; x < a.G * D; x += kConsumerWarps * 32) {
+      const int h = x / D, dd = x % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, stats[(w * NH + h) * 2]);
+      const float base = M == -INFINITY ? 0.f : M;
+      float o = 0.f, L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float f = ex2(stats[(w * NH + h) * 2] - base);
+        o += comb[(w * NH + h) * D + dd] * f;
+        L += stats[(w * NH + h) * 2 + 1] * f;
+      }
+      const int64_t pidx = static_cast<int64_t>(unit) * a.G + h;
+      a.part_o[pidx * D + dd] = o;
+      if (dd == 0) {
+        a.part_ml[pidx * 2 + 0] = M;
+        a.part_ml[pidx * 2 + 1] = L;
+      }
+    }
+    if (!consumer_sync_and(alive)) break;
+  }
+}
+
+// One warp per (b, h): combine the splits of its row.
+template <int D>
+__global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a) {
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= a.B * a.Hq) return;
+  const int b = wid / a.Hq, h = wid % a.Hq;
+  const int g = h / a.G, hl = h % a.G;
+  const int row = b * a.Hkv + g;
+  constexpr int PER = D / 32;
+  float M = -INFINITY;
+  for (int s = 0; s < a.splits; ++s) {
+    const int64_t pidx = static_cast<int64_t>(row * a.splits + s) * a.G + hl;
+    M = fmaxf(M, a.part_ml[pidx * 2]);
+  }
+  const float base = M == -INFINITY ? 0.f : M;
+  float o[PER];
+#pragma unroll
+  for (int q = 0; q < PER; ++q) o[q] = 0.f;
+  float L = 0.f;
+  for (int s = 0; s < a.splits; ++s) {
+    const int64_t pidx = static_cast<int64_t>(row * a.splits + s) * a.G + hl;
+    const float f = ex2(a.part_ml[pidx * 2] - base);
+    L += a.part_ml[pidx * 2 + 1] * f;
+    const float* po = a.part_o + pidx * D;
+#pragma unroll
+    for (int q = 0; q < PER; ++q) o[q] += po[lane + 32 * q] * f;
+  }
+  const float inv = L > 0.f ? 1.0f / L : 0.f;
+  const int64_t obase = (static_cast<int64_t>(b) * a.Hq + h) * D;
+  __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o);
+#pragma unroll
+  for (int q = 0; q < PER; ++q) {
+    const float v = o[q] * inv;
+    ob[obase + lane + 32 * q] = __float2bfloat16_rn(v);
+    if (a.o_f32) a.o_f32[obase + lane + 32 * q] = v;
+  }
+  if (lane == 0) {
+    // natural-log LSE from the log2-domain running max and sum
+    a.lse[static_cast<int64_t>(b) * a.Hq + h] =
+        L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+  }
+}
+
+template <int D, int NT>
+cudaError_t launch_dn(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                      int num_units, int num_sms, cudaStream_t s) {
+  const int smem = DecodeSmem<D, NT>::kTotal;
+  auto kern = decode_attn_kernel<D, NT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int grid = num_units < num_sms ? num_units : num_sms;
+  if (grid > 0) kern<<<grid, kThreads, smem, s>>>(a, tk, tv, num_units);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int warps = a.B * a.Hq;
+  lse_merge_kernel<D><<<(warps * 32 + 255) / 256, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+void decode_split_plan(int rows, int max_kept, int num_sms, int* splits, int* split_len) {
+  // minimise (units per CTA, rounded up) * (blocks per unit + per-unit overhead)
+  const double overhead = 2.0;
+  int best_len = max_kept > 0 ? max_kept : 1;
+  double best = 1e300;
+  for (int len = 1; len <= (max_kept > 0 ? max_kept : 1); ++len) {
+    const int sp = (max_kept + len - 1) / len;
+    const long units = static_cast<long>(rows) * (sp > 0 ? sp : 1);
+    const long waves = (units + num_sms - 1) / num_sms;
+    const double cost = static_cast<double>(waves) * (len + overhead);
+    if (cost < best - 1e-9) {
+      best = cost;
+      best_len = len;
+    }
+  }
+  *split_len = best_len;
+  *splits = max_kept > 0 ? (max_kept + best_len - 1) / best_len : 1;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                          int num_units, int num_sms, cudaStream_t s) {
+  const int NT = a.G > 8 ? 2 : 1;
+  if (a.d == 128) {
+    return NT == 1 ? launch_dn<128, 1>(a, tk, tv, num_units, num_sms, s)
+                   : launch_dn<128, 2>(a, tk, tv, num_units, num_sms, s);
+  }
+  return NT == 1 ? launch_dn<64, 1>(a, tk, tv, num_units, num_sms, s)
+                 : launch_dn<64, 2>(a, tk, tv, num_units, num_sms, s);
+}
+
+}  // namespace bsa

@@ -1,0 +1,145 @@
+// Prefill block scorer.
+//
+// For every (sequence b, kv head g, query block i) and key block j < i:
+//   S[b,g,i,j] = idx_scale * max_{tq in block i, tq < T; tk in block j}
+//                sum_{h in group g} w_h ReLU(q_idx[b,h,tq] . k_idx[b,g,tk])
+// (SpotAttention, Methodology §1: weighted-ReLU selector score, run as one
+//  matrix product; the O(T^2) cost of this step is the point SparDA,
+//  "Problem statement", makes about block selection.)
+//
+// Design: one CTA (4 warps) per query-block row; warp w owns query tokens
+// [16w, 16w+16). Its index-query fragments stay in registers for the whole row:
+// mma.m16n8k16 with rows = (head pair, 8 query tokens), columns = 8 key tokens,
+// K = r = 16 (same dim relabelling as the decode scorer, so each lane loads one
+// 8-byte run per token). A lane then holds every head's dot product for its
+// (tq, tk) pairs, so ReLU, weights and the head sum need no shuffles; the 64x64
+// tile max is a per-lane running max plus one warp reduction, and the four
+// warps' maxima are combined through shared memory in batches of key blocks.
+#include "bsa_common.cuh"
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kBatch = 32;  // key blocks per shared-memory combine
+
+template <int HP>  // head pairs = ceil(G / 2)
+__global__ void __launch_bounds__(kWarps * 32) score_prefill_kernel(const ScorePrefillArgs a) {
+  __shared__ float pm[kWarps][kBatch];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int BH = a.B * a.Hkv;
+  const int i = a.nqb - 1 - static_cast<int>(blockIdx.x) / BH;  // heavy rows first
+  const int bg = static_cast<int>(blockIdx.x) % BH;
+  const int b = bg / a.Hkv, g = bg % a.Hkv;
+  if (i <= 0) return;
+
+  // query fragments: tq group tg (8 tokens), head pair hp
+  uint32_t aq[2][HP][4];
+  float w[HP][2];
+  const char* qbase = static_cast<const char*>(a.q_idx);
+  const float dflt = 1.0f / static_cast<float>(a.G);
+#pragma unroll
+  for (int hp = 0; hp < HP; ++hp) {
+    const int h0 = 2 * hp, h1 = 2 * hp + 1;
+    w[hp][0] = h0 < a.G ? (a.head_w ? a.head_w[g * a.G + h0] : dflt) : 0.f;
+    w[hp][1] = h1 < a.G ? (a.head_w ? a.head_w[g * a.G + h1] : dflt) : 0.f;
+#pragma unroll
+    for (int tg = 0; tg < 2; ++tg) {
+      const int tq = i * kBlock + 16 * warp + 8 * tg + gid;
+      const bool tv = tq < a.T;
+      uint2 x0 = make_uint2(0u, 0u), x1 = make_uint2(0u, 0u);
+      if (tv && h0 < a.G)
+        x0 = *reinterpret_cast<const uint2*>(
+            qbase + (((static_cast<int64_t>(b) * a.Hq + g * a.G + h0) * a.T + tq) * kR + 4 * tig) * 2);
+      if (tv && h1 < a.G)
+        x1 = *reinterpret_cast<const uint2*>(
+            qbase + (((static_cast<int64_t>(b) * a.Hq + g * a.G + h1) * a.T + tq) * kR + 4 * tig) * 2);
+      aq[tg][hp][0] = x0.x;
+      aq[tg][hp][1] = x1.x;
+      aq[tg][hp][2] = x0.y;
+      aq[tg][hp][3] = x1.y;
+    }
+  }
+  // query tokens of this lane that exist (a ragged last query block)
+  const bool q0v = i * kBlock + 16 * warp + gid < a.T;
+  const bool q1v = i * kBlock + 16 * warp + 8 + gid < a.T;
+
+  const char* kbase = static_cast<const char*>(a.kidx.base);
+  float* out = a.scores + (static_cast<int64_t>(bg) * a.nqb + i) * a.nqb;
+
+  for (int j0 = 0; j0 < i; j0 += kBatch) {
+    const int jn = min(kBatch, i - j0);
+    for (int jj = 0; jj < jn; ++jj) {
+      const int j = j0 + jj;
+      int64_t phys = j;
+      bool ok = true;
+      if (a.kidx.page_table != nullptr) {
+        phys = a.kidx.page_table[static_cast<int64_t>(b) * a.kidx.pt_stride + j];
+        ok = phys >= 0 && phys < a.kidx.num_pages;
+      }
+      const int64_t off = static_cast<int64_t>(b) * a.kidx.seq_stride + phys * a.kidx.block_stride +
+                          static_cast<int64_t>(g) * a.kidx.head_stride;
+      ok = ok && off >= 0 && off + kBlock * kR <= a.kidx.extent;
+      float mx = 0.f;
+      if (ok) {
+        const char* kb = kbase + off * 2;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          const uint2 kv = *reinterpret_cast<const uint2*>(kb + (nt * 8 + gid) * 32 + tig * 8);
+#pragma unroll
+          for (int tg = 0; tg < 2; ++tg) {
+            float u0 = 0.f, u1 = 0.f;
+#pragma unroll
+            for (int hp = 0; hp < HP; ++hp) {
+              float c[4] = {0.f, 0.f, 0.f, 0.f};
+              mma_bf16(c, aq[tg][hp], kv.x, kv.y);
+              u0 = fmaf(w[hp][0], fmaxf(c[0], 0.f), u0);
+              u0 = fmaf(w[hp][1], fmaxf(c[2], 0.f), u0);
+              u1 = fmaf(w[hp][0], fmaxf(c[1], 0.f), u1);
+              u1 = fmaf(w[hp][1], fmaxf(c[3], 0.f), u1);
+            }
+            const bool qv = tg == 0 ? q0v : q1v;
+            if (qv) mx = fmaxf(mx, fmaxf(u0, u1));
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      } else {
+        mx = -INFINITY;
+        if (lane == 0 && warp == 0) report(a.status, BSA_DEV_BAD_PAGE);
+      }
+      if (lane == 0) pm[warp][jj] = mx;
+    }
+    __syncthreads();
+    if (threadIdx.x < jn) {
+      float m = pm[0][threadIdx.x];
+#pragma unroll
+      for (int ww = 1; ww < kWarps; ++ww) m = fmaxf(m, pm[ww][threadIdx.x]);
+      const float sc = a.idx_scale * m;
+      out[j0 + threadIdx.x] = sc;
+      if (!isfinite(sc)) report(a.status, BSA_DEV_NONFINITE);
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_score_prefill(const ScorePrefillArgs& a, int num_sms, cudaStream_t s) {
+  (void)num_sms;
+  const int rows = a.B * a.Hkv * a.nqb;
+  if (rows <= 0) return cudaSuccess;
+  const int HP = (a.G + 1) / 2;
+  switch (HP) {
+    case 1: score_prefill_kernel<1><<<rows, kWarps * 32, 0, s>>>(a); break;
+    case 2: score_prefill_kernel<2><<<rows, kWarps * 32, 0, s>>>(a); break;
+    case 4: score_prefill_kernel<4><<<rows, kWarps * 32, 0, s>>>(a); break;
+    case 8: score_prefill_kernel<8><<<rows, kWarps * 32, 0, s>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

@@ -1,0 +1,348 @@
+// Block selection: sinks + local window + dynamic top-p over the residual
+// candidates, capped at k_max, floored at k_min; ties to the lower block id.
+// (SpotAttention, Methodology §3: reserved sink prefix and recency suffix,
+//  nucleus selection on the residual distribution until the cumulative mass
+//  reaches p, floor K_min; RTPurbo, Methodology §3 (dynamic top-p) and §5
+//  (histogram thresholding instead of a sort); HGA, Central mechanism §2 for
+//  the prefill diagonal block.)
+//
+// One CTA per row: decode row = (b, g); prefill row = (b, g, query block i).
+// The candidates form one contiguous id range [c0, c1) in both phases. Steps:
+//  1. keys: 32-bit order keys (smaller key = higher score; -0 folded into +0,
+//     NaN last) staged in shared memory; M = max score over the candidates;
+//  2. radix select (4 passes x 8 bits, warp-aggregated shared-memory histograms,
+//     integer counts only, so deterministic) of the key of the Kcap-th candidate,
+//     Kcap = the largest dynamic count the caps allow; equal keys are taken in
+//     ascending id order via a block-wide scan;
+//  3. when 0 < p < 1: the Kcap winners are sorted by (key, id) with a bitonic
+//     sort, their masses exp(S - M) are prefix-summed in fp64 along that order
+//     (fixed order, deterministic) and the first prefix reaching p * Z is cut,
+//     Z = sum of exp(S - M) over all candidates (fp64, fixed reduction tree);
+//  4. kept list = [0, c0) ++ ascending dynamic ids ++ [c1, end), -1 padded.
+#include "bsa_common.cuh"
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace {
+
+constexpr int kHistCopies = 8;
+
+BSA_DEVFN uint32_t order_key(float s) {
+  if (s != s) return 0xffffffffu;           // NaN: lowest priority
+  s = s + 0.0f;                               // -0 -> +0
+  uint32_t u = __float_as_uint(s);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending in s
+  return ~u;                                  // ascending key = descending score
+}
+
+__host__ __device__ __forceinline__ int skew(int i) { return i + (i >> 5); }
+
+// Deterministic block reductions / scans (fixed tree for a fixed NT).
+template <int NT, typename T, typename Op>
+BSA_DEVFN T block_allreduce(T v, T* scratch, Op op) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  T r = scratch[0];
+  for (int w = 1; w < NT / 32; ++w) r = op(r, scratch[w]);
+  __syncthreads();
+  return r;
+}
+
+// Exclusive scan of one value per thread in thread order; returns the prefix, sets total.
+template <int NT, typename T>
+BSA_DEVFN T block_exscan(T v, T* scratch, T& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  T inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    T n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  __syncthreads();
+  if (lane == 31) scratch[warp] = inc;
+  __syncthreads();
+  T base = T(0);
+  for (int w = 0; w < warp; ++w) base += scratch[w];
+  T tot = T(0);
+  for (int w = 0; w < NT / 32; ++w) tot += scratch[w];
+  total = tot;
+  __syncthreads();
+  return base + inc - v;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_nc, int sort_n) {
+  constexpr int NW = NT / 32;
+  extern __shared__ __align__(16) unsigned char smem[];
+  // layout: [sort buffer: sort_n u64][keys: skew(max_nc) u32][hist: copies*256 u32]
+  //         [flags: (max_nc+31)/32 u32][scratch]
+  uint64_t* sbuf = reinterpret_cast<uint64_t*>(smem);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sbuf + sort_n);
+  uint32_t* hist = keys + skew(max_nc) + 1;
+  uint32_t* flags = hist + kHistCopies * 256;
+  const int nflag_words = (max_nc + 31) / 32;
+  __shared__ double dscr[NW];
+  __shared__ uint32_t s_bucket_info[2];
+  __shared__ int s_hit;
+  __shared__ float s_fscr[NW];
+  __shared__ int s_iscr[NW];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = blockIdx.x;
+
+  // ---- row geometry -------------------------------------------------------
+  int nbr, c0, c1;
+  const float* S;
+  int32_t* kept;
+  int32_t* kcount;
+  if (a.phase == BSA_PHASE_DECODE) {
+    const int b = row / a.Hkv;
+    int Tb = a.seq_lens ? a.seq_lens[b] : a.T;
+    Tb = Tb < 0 ? 0 : (Tb > a.T ? a.T : Tb);
+    nbr = (Tb + kBlock - 1) / kBlock;
+    c0 = min(a.n_sink, nbr);
+    c1 = max(c0, nbr - a.n_local);
+    S = a.scores + static_cast<int64_t>(row) * a.nb_max;
+  } else {
+    const int i = row % a.nqb;
+    nbr = i + 1;
+    c0 = min(a.n_sink, i);
+    c1 = max(c0, i - a.n_local);
+    S = a.scores + static_cast<int64_t>(row) * a.nqb;
+  }
+  kept = a.kept + static_cast<int64_t>(row) * a.max_kept;
+  kcount = a.kept_count + row;
+  const int nC = c1 - c0;
+
+  const float ph = a.p;
+  int kcap;  // largest number of dynamic blocks the caps allow
+  const int kminC = min(a.k_min, nC);
+  if (ph <= 0.f)
+    kcap = kminC;
+  else
+    kcap = max(min(a.k_max, nC), kminC);
+  const bool need_mass = (ph > 0.f) && (ph < 1.f) && kcap > 0;
+
+  // ---- 1. keys and max ------------------------------------------------------
+  float lmax = -INFINITY;
+  for (int t = tid; t < nC; t += NT) {
+    const float s = S[c0 + t];
+    keys[skew(t)] = order_key(s);
+    if (s == s) lmax = fmaxf(lmax, s);
+  }
+  for (int w = tid; w < nflag_words; w += NT) flags[w] = 0u;
+  const float M = block_allreduce<NT>(lmax, s_fscr, [](float x, float y) { return fmaxf(x, y); });
+
+  // blocked ownership for the scans: thread t owns [t*E, min(nC, (t+1)*E))
+  const int E = (nC + NT - 1) / NT;
+  const int seg0 = min(nC, tid * E), seg1 = min(nC, seg0 + E);
+
+  int kdyn = 0;
+  if (kcap > 0 && kcap < nC) {
+    // ---- 2. radix select of the kcap-th key ------------------------------------
+    uint32_t prefix = 0u, pmask = 0u;
+    int rem = kcap;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int x = tid; x < kHistCopies * 256; x += NT) hist[x] = 0u;
+      __syncthreads();
+      uint32_t* h = hist + (warp % kHistCopies) * 256;
+      for (int t0 = 0; t0 < nC; t0 += NT) {
+        const int t = t0 + tid;
+        uint32_t digit = 256u;
+        if (t < nC) {
+          const uint32_t k = keys[skew(t)];
+          if ((k & pmask) == prefix) digit = (k >> shift) & 255u;
+        }
+        const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+        if (digit < 256u && lane == __ffs(peers) - 1) atomicAdd(&h[digit], __popc(peers));
+      }
+      __syncthreads();
+      for (int x = tid; x < 256; x += NT) {
+        uint32_t tot = 0;
+        for (int c = 0; c < kHistCopies; ++c) tot += hist[c * 256 + x];
+        hist[x] = tot;  // copy 0 now holds totals (other copies no longer needed)
+      }
+      __syncthreads();
+      if (warp == 0) {
+        uint32_t part = 0;
+        for (int q = 0; q < 8; ++q) part += hist[lane * 8 + q];
+        uint32_t inc = part;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += n;
+        }
+        const uint32_t exc = inc - part;
+        const bool here = (exc < static_cast<uint32_t>(rem)) && (inc >= static_cast<uint32_t>(rem));
+        if (here) {
+          uint32_t c = exc;
+          int bsel = lane * 8;
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t hq = hist[lane * 8 + q];
+            if (c + hq >= static_cast<uint32_t>(rem)) {
+              bsel = lane * 8 + q;
+              break;
+            }
+            c += hq;
+          }
+          s_bucket_info[0] = static_cast<uint32_t>(bsel);
+          s_bucket_info[1] = c;  // count strictly below the bucket
+        }
+      }
+      __syncthreads();
+      prefix |= s_bucket_info[0] << shift;
+      pmask |= 255u << shift;
+      rem -= static_cast<int>(s_bucket_info[1]);
+      __syncthreads();
+    }
+    // keys < prefix are in; among keys == prefix take the `rem` lowest ids
+    int neq = 0;
+    for (int t = seg0; t < seg1; ++t) neq += (keys[skew(t)] == prefix);
+    int tot_eq;
+    int eq_base = block_exscan<NT>(neq, s_iscr, tot_eq);
+    for (int t = seg0; t < seg1; ++t) {
+      const uint32_t k = keys[skew(t)];
+      bool in = k < prefix;
+      if (k == prefix) in = (eq_base++ < rem);
+      if (in) atomicOr(&flags[t >> 5], 1u << (t & 31));
+    }
+    kdyn = kcap;
+  } else if (kcap > 0) {  // every candidate is within the caps
+    for (int t = tid; t < nC; t += NT) atomicOr(&flags[t >> 5], 1u << (t & 31));
+    kdyn = nC;
+  }
+  __syncthreads();
+
+  // ---- 3. top-p cut inside the kcap winners ------------------------------------
+  if (need_mass) {
+    // total mass over the candidates (fp64, fixed order)
+    double z = 0.0;
+    const double Md = static_cast<double>(M);
+    const bool all_inf = !(M > -INFINITY);
+    for (int t = seg0; t < seg1; ++t) {
+      const float s = S[c0 + t];
+      z += all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
+    }
+    double Z = block_allreduce<NT>(z, dscr, [](double x, double y) { return x + y; });
+    // compact winners in id order, then sort by (key, id)
+    int nsel = 0;
+    for (int t = seg0; t < seg1; ++t) nsel += (flags[t >> 5] >> (t & 31)) & 1u;
+    int tot;
+    int pos = block_exscan<NT>(nsel, s_iscr, tot);
+    for (int t = seg0; t < seg1; ++t)
+      if ((flags[t >> 5] >> (t & 31)) & 1u)
+        sbuf[pos++] = (static_cast<uint64_t>(keys[skew(t)]) << 32) | static_cast<uint32_t>(t);
+    for (int x = kdyn + tid; x < sort_n; x += NT) sbuf[x] = ~0ull;
+    __syncthreads();
+    for (int kk = 2; kk <= sort_n; kk <<= 1) {
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        for (int x = tid; x < sort_n; x += NT) {
+          const int y = x ^ j;
+          if (y > x) {
+            const uint64_t u = sbuf[x], v = sbuf[y];
+            const bool asc = (x & kk) == 0;
+            if ((u > v) == asc) {
+              sbuf[x] = v;
+              sbuf[y] = u;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    // inclusive fp64 prefix of masses along the sorted order
+    const int E2 = (kdyn + NT - 1) / NT;
+    const int q0 = min(kdyn, tid * E2), q1 = min(kdyn, q0 + E2);
+    double loc = 0.0;
+    for (int x = q0; x < q1; ++x) {
+      const float s = S[c0 + static_cast<int>(sbuf[x] & 0xffffffffu)];
+      loc += all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
+    }
+    double dtot;
+    double run = block_exscan<NT>(loc, dscr, dtot);
+    if (tid == 0) s_hit = 0x7fffffff;
+    __syncthreads();
+    const double target = static_cast<double>(ph) * Z;
+    for (int x = q0; x < q1; ++x) {
+      const float s = S[c0 + static_cast<int>(sbuf[x] & 0xffffffffu)];
+      run += all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
+      if (run >= target) {
+        atomicMin(&s_hit, x);
+        break;
+      }
+    }
+    __syncthreads();
+    const int capC = min(a.k_max, nC);
+    const int k = (s_hit != 0x7fffffff) ? max(min(s_hit + 1, capC), kminC) : kdyn;
+    // re-flag the first k of the order
+    for (int w = tid; w < nflag_words; w += NT) flags[w] = 0u;
+    __syncthreads();
+    for (int x = tid; x < k; x += NT) {
+      const int t = static_cast<int>(sbuf[x] & 0xffffffffu);
+      atomicOr(&flags[t >> 5], 1u << (t & 31));
+    }
+    kdyn = k;
+    __syncthreads();
+  }
+
+  // ---- 4. kept list ----------------------------------------------------------
+  int nsel = 0;
+  for (int t = seg0; t < seg1; ++t) nsel += (flags[t >> 5] >> (t & 31)) & 1u;
+  int tot;
+  int pos = block_exscan<NT>(nsel, s_iscr, tot);
+  for (int t = seg0; t < seg1; ++t)
+    if ((flags[t >> 5] >> (t & 31)) & 1u) kept[c0 + pos++] = c0 + t;
+  for (int x = tid; x < c0; x += NT) kept[x] = x;
+  const int nlocal = nbr - c1;
+  for (int x = tid; x < nlocal; x += NT) kept[c0 + tot + x] = c1 + x;
+  const int count = c0 + tot + nlocal;
+  for (int x = count + tid; x < a.max_kept; x += NT) kept[x] = -1;
+  if (tid == 0) *kcount = count;
+}
+
+int pow2_at_least(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+template <int NT>
+cudaError_t launch_nt(const SelectArgs& a, int rows, int max_nc, cudaStream_t s) {
+  const int kcap_max = max(min(a.k_max, max_nc), min(a.k_min, max_nc));
+  const int sort_n = pow2_at_least(max(kcap_max, 2));
+  const int nflag_words = (max_nc + 31) / 32;
+  size_t smem = static_cast<size_t>(sort_n) * 8 + (static_cast<size_t>(skew(max_nc)) + 1) * 4 +
+                kHistCopies * 256 * 4 + (nflag_words + 1) * 4;
+  smem = (smem + 15) & ~static_cast<size_t>(15);
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<NT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  select_kernel<NT><<<rows, NT, smem, s>>>(a, max_nc, sort_n);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
+  int rows, max_nc;
+  if (a.phase == BSA_PHASE_DECODE) {
+    rows = a.B * a.Hkv;
+    max_nc = a.nb_max;
+  } else {
+    rows = a.B * a.Hkv * a.nqb;
+    max_nc = a.nqb;
+  }
+  if (rows <= 0) return cudaSuccess;
+  max_nc = max(max_nc, 1);
+  if (max_nc <= 2048) return launch_nt<256>(a, rows, max_nc, s);
+  if (max_nc <= 8192) return launch_nt<512>(a, rows, max_nc, s);
+  return launch_nt<1024>(a, rows, max_nc, s);
+}
+
+}  // namespace bsa

@@ -1,0 +1,163 @@
+/*
+ * bsa.h - C ABI of the dynamic block-sparse attention library for long-context
+ * decode and prefill on NVIDIA B200 (sm_100a). Shared library: libbsa.so.
+ *
+ * The method (cited by page title and section of the gist.science summaries):
+ *   1. Score. Every 64-token KV block gets a score from a low-dimensional index
+ *      (r = 16 index keys and queries, RTPurbo "Full Attention Strikes Back",
+ *      Methodology §2): per token t, u_t = idx_scale * sum_h w_h ReLU(q_idx[h] . k_idx[t])
+ *      over the query heads h of the kv group (SpotAttention, Methodology §1);
+ *      the block score is the max of u over the block's tokens (prefill: over the
+ *      query block x key block tile).
+ *   2. Select. Keep the sink blocks and the local (recency) blocks; among the
+ *      remaining candidate blocks keep the shortest prefix, in order of score
+ *      (ties to the lower block id), whose softmax mass over the candidates
+ *      reaches p, capped at k_max and floored at k_min (SpotAttention,
+ *      Methodology §3; RTPurbo, Methodology §3). Prefill also keeps the current
+ *      (diagonal) block (HGA, Central mechanism §2).
+ *   3. Attend. Exact softmax attention over the token-level K/V of the kept
+ *      blocks only (HGA, Central mechanism §4), causal within the diagonal block
+ *      in prefill.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer argument except `stream` is a DEVICE pointer unless stated.
+ *     The caller owns all memory; the library never allocates, frees or
+ *     synchronizes, and keeps no global state apart from per-device launch
+ *     parameters read once (SM count) and the TMA encode entry point.
+ *   - All work is enqueued on `stream` (a cudaStream_t passed as void*; NULL =
+ *     the legacy default stream). Calls return after the launch, not after the
+ *     work; they are re-entrant on distinct output and workspace buffers.
+ *   - Host-checkable errors (shapes, null pointers, alignment) return a status
+ *     and launch nothing. Data errors found on the device (page id out of range,
+ *     kept id out of range, non-finite score, a bounded wait that gave up) are
+ *     OR-ed as BSA_DEV_* bits into *dev_status (int32, may be NULL); kernels
+ *     never trap. A launch failure returns BSA_ERR_CUDA.
+ *   - Supported shapes: block = 64, r = 16, d in {64, 128}, Hq % Hkv == 0,
+ *     G = Hq / Hkv in {1, 2, 4, 8, 16}, k_min <= k_max <= 8192, contexts up to
+ *     32768 blocks (2^21 tokens). bf16 tensors must be 16-byte aligned.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1, /* bad argument; nothing launched */
+  BSA_ERR_UNSUPPORTED = 2, /* valid but outside the supported shapes; nothing launched */
+  BSA_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than bsa_workspace_size() */
+  BSA_ERR_CUDA = 4         /* a CUDA call or kernel launch failed */
+} bsa_status_t;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define BSA_DEV_BAD_PAGE 0x1   /* page id outside [0, num_pages) or block beyond extent: skipped */
+#define BSA_DEV_BAD_KEPT 0x2   /* kept block id outside [0, nb): skipped */
+#define BSA_DEV_NONFINITE 0x4  /* a block score was +-inf or NaN */
+#define BSA_DEV_TIMEOUT 0x8    /* a bounded wait inside a kernel gave up; outputs invalid */
+#define BSA_DEV_FP16_RANGE 0x10 /* prefill: a V value outside the fp16 range */
+
+typedef enum { BSA_PHASE_DECODE = 0, BSA_PHASE_PREFILL = 1 } bsa_phase_t;
+
+typedef enum { BSA_OP_SCORE = 0, BSA_OP_SELECT = 1, BSA_OP_DECODE = 2, BSA_OP_PREFILL = 3 } bsa_op_t;
+
+/* Addressing of one bf16 cache tensor (K, V or index keys), contiguous or paged.
+ * Token t of sequence b, kv head g starts at element
+ *     b*seq_stride + phys*block_stride + g*head_stride + (t % 64)*width
+ * from `base`, where phys = page_table[b*page_table_stride + t/64] when
+ * page_table != NULL and phys = t/64 otherwise, and width = d (K, V) or r
+ * (index keys). The 64 rows of one block of one head are contiguous.
+ * Contiguous [B, Hkv, T, w]: seq_stride = Hkv*T*w, block_stride = 64*w,
+ * head_stride = T*w. Paged pool [P, Hkv, 64, w]: seq_stride = 0,
+ * block_stride = Hkv*64*w, head_stride = 64*w, num_pages = P.
+ * `extent` = number of elements addressable from base; every block read is
+ * checked against it (and page ids against num_pages). */
+typedef struct {
+  const void* base;
+  int64_t seq_stride;
+  int64_t block_stride;
+  int64_t head_stride;
+  const int32_t* page_table; /* [B, page_table_stride] or NULL */
+  int32_t page_table_stride;
+  int32_t num_pages;         /* used when page_table != NULL */
+  int64_t extent;
+} bsa_cache_t;
+
+/* Problem description shared by all entry points. */
+typedef struct {
+  int32_t phase;            /* bsa_phase_t */
+  int32_t B, Hq, Hkv, d, r, block;
+  int32_t T;                /* decode: capacity, every seq_lens[b] <= T; prefill: sequence length */
+  const int32_t* seq_lens;  /* decode: device [B] tokens per sequence (>= 0), or NULL = T */
+  int32_t n_sink;           /* sink blocks kept [0, n_sink) */
+  int32_t n_local;          /* local blocks kept: decode [nb-n_local, nb), prefill [i-n_local, i) */
+  int32_t k_max;            /* cap on dynamically selected blocks */
+  int32_t k_min;            /* floor on dynamically selected blocks (<= k_max) */
+  float p;                  /* top-p threshold; <= 0: none, >= 1: all (then capped) */
+  float idx_scale;          /* index score scale; 0 = 1/sqrt(r) */
+  float attn_scale;         /* softmax scale; 0 = 1/sqrt(d) */
+  const float* head_w;      /* device [Hq] non-negative index-head weights, or NULL = 1/G */
+} bsa_problem_t;
+
+/* Length of one kept list: decode n_sink + n_local + k_max; prefill
+ * 1 + n_sink + n_local + k_max. Unused slots of a list hold -1. */
+int32_t bsa_max_kept(const bsa_problem_t* prob);
+
+/* Workspace bytes `op` needs for `prob` (0 when none). Host only. */
+bsa_status_t bsa_workspace_size(const bsa_problem_t* prob, int32_t op, size_t* bytes);
+
+/* Step 1, block scores (SpotAttention, Methodology §1; RTPurbo, Methodology §2).
+ * decode:  q_idx [B, Hq, r] bf16 -> block_scores [B, Hkv, nb] fp32, nb = ceil(T/64);
+ *          entries j >= ceil(seq_lens[b]/64) are set to -inf.
+ * prefill: q_idx [B, Hq, T, r] bf16 -> block_scores [B, Hkv, nqb, nqb] fp32,
+ *          nqb = ceil(T/64); entry [i, j] written for j < i only.
+ * k_idx addresses index keys (width r). */
+bsa_status_t bsa_score_blocks(const bsa_problem_t* prob, const void* q_idx, bsa_cache_t k_idx,
+                              float* block_scores, int32_t* dev_status, void* stream);
+
+/* Step 2, selection (SpotAttention, Methodology §3; RTPurbo, Methodology §3 and
+ * §5 - histogram thresholding without a sort over all blocks).
+ * decode:  rows (b, g): kept [B, Hkv, max_kept] ascending block ids, -1 padded;
+ *          kept_count [B, Hkv].
+ * prefill: rows (b, g, i): kept [B, Hkv, nqb, max_kept], kept_count [B, Hkv, nqb];
+ *          candidates are key blocks j < i outside the reserved set. */
+bsa_status_t bsa_select_top_p(const bsa_problem_t* prob, const float* block_scores,
+                              int32_t* kept, int32_t* kept_count, int32_t* dev_status,
+                              void* stream);
+
+/* Step 3, decode attention over the kept blocks (HGA, Central mechanism §4):
+ * split-K flash-decode with an LSE merge.
+ * q [B, Hq, d] bf16; k, v caches (width d); kept/kept_count from step 2.
+ * Outputs: o [B, Hq, d] bf16, lse [B, Hq] fp32 (natural log; -inf and o = 0 when
+ * a row has no visible token), o_f32 [B, Hq, d] fp32 or NULL. Workspace: see
+ * bsa_workspace_size(BSA_OP_DECODE). */
+bsa_status_t bsa_decode(const bsa_problem_t* prob, const void* q, bsa_cache_t k, bsa_cache_t v,
+                        const int32_t* kept, const int32_t* kept_count, void* o, float* lse,
+                        float* o_f32, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, void* stream);
+
+/* Step 3, block-sparse causal prefill attention (HGA, Central mechanism §4).
+ * q [B, Hq, T, d] bf16; k, v caches (width d) holding the T prompt tokens;
+ * kept/kept_count from step 2 (prefill). Outputs: o [B, Hq, T, d] bf16,
+ * lse [B, Hq, T] fp32, o_f32 [B, Hq, T, d] fp32 or NULL. V values must lie in
+ * the fp16 range (|v| <= 65504): P.V runs on fp16 tensor-core operands. */
+bsa_status_t bsa_prefill(const bsa_problem_t* prob, const void* q, bsa_cache_t k, bsa_cache_t v,
+                         const int32_t* kept, const int32_t* kept_count, void* o, float* lse,
+                         float* o_f32, void* workspace, size_t workspace_bytes,
+                         int32_t* dev_status, void* stream);
+
+/* Static description of a status code. */
+const char* bsa_status_string(bsa_status_t status);
+
+/* Last CUDA error string seen by this thread's most recent BSA_ERR_CUDA (or ""). */
+const char* bsa_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H */

@@ -1,0 +1,226 @@
+"""Parity helpers: run the fp64 oracle on rows of a generated workload and compare
+the CUDA path's outputs with it (test infrastructure).
+
+Bars (the decode/prefill accuracy statement of the method's target):
+* block selection identical, except a near-tie at the top-p / K_max boundary:
+  the oracle's competing masses differ by less than 1e-6 relative; such rows are
+  reported as ties and their attention is re-checked against the oracle run on
+  the device's kept set;
+* attention output (fp32 copy of the normalised output) max-abs <= 2e-3 and
+  relative L2 <= 1e-3 against the oracle; the bf16 output equals the
+  round-to-nearest-even of that fp32 copy bit for bit; |LSE error| <= 1e-4;
+* block scores (fp32 on the device) within 1e-5 relative of the oracle's.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from oracle import bsa_oracle as O
+
+TIE_REL = 1e-6
+O_MAX_ABS = 2e-3
+O_REL_L2 = 1e-3
+LSE_ABS = 1e-4
+SCORE_REL = 1e-5
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+# ------------------------------------------------------------------ tie rule
+def classify_selection(sel: O.Selection, kept_dev, tol=TIE_REL):
+    """'exact' | 'tie' | 'mismatch: ...' for a device kept list against the oracle."""
+    kept_dev = [int(x) for x in kept_dev]
+    if sorted(kept_dev) != kept_dev or len(set(kept_dev)) != len(kept_dev):
+        return "mismatch: device list not strictly ascending"
+    R, C = set(sel.reserved), set(sel.candidates)
+    Kd = set(kept_dev)
+    if not R <= Kd:
+        return f"mismatch: reserved blocks missing {sorted(R - Kd)}"
+    if not Kd <= (R | C):
+        return f"mismatch: blocks outside the row {sorted(Kd - R - C)}"
+    Dd = Kd - R
+    k = sel.k
+    Do = set(sel.order[:k])
+    if Dd == Do:
+        return "exact"
+    pos = {j: t for t, j in enumerate(sel.order)}
+    mass = {j: sel.mass[pos[j]] for j in sel.order}
+    kd = len(Dd)
+    if kd == k:
+        mb = sel.mass[k - 1]
+        bad = [j for j in (Do ^ Dd) if abs(mass[j] - mb) > tol * mb]
+        return "tie" if not bad else f"mismatch: blocks {sorted(Do ^ Dd)} differ (masses {[mass[j] for j in sorted(Do ^ Dd)]}, boundary {mb})"
+    if abs(kd - k) == 1:
+        kk = min(k, kd)
+        cum = sel.cum[kk - 1] if kk >= 1 else 0.0
+        return ("tie-count", kk, cum, kd)
+    return f"mismatch: {kd} dynamic blocks on the device, {k} in the oracle"
+
+
+def selection_verdict(sel: O.Selection, kept_dev, p: float, tol=TIE_REL):
+    r = classify_selection(sel, kept_dev, tol)
+    if isinstance(r, tuple):       # count differs by one: cumulative mass at the cut ~ p
+        _, kk, cum, kd = r
+        ph = O.p_hat(p)
+        if abs(cum - ph) > tol * ph:
+            return f"mismatch: count {kd} vs {sel.k} and cumulative {cum} not within tie of {ph}"
+        Dd = set(int(x) for x in kept_dev) - set(sel.reserved)
+        ref = set(sel.order[:kd])
+        pos = {j: t for t, j in enumerate(sel.order)}
+        mb = sel.mass[kd - 1] if kd >= 1 else 0.0
+        bad = [j for j in (ref ^ Dd) if abs(sel.mass[pos[j]] - mb) > tol * max(mb, 1e-300)]
+        return "tie" if not bad else f"mismatch: count tie but blocks {sorted(ref ^ Dd)} differ"
+    return r
+
+
+# ------------------------------------------------------------------ attention bars
+def attention_errors(o_f32_dev, o_bf16_dev, lse_dev, o_ref, lse_ref):
+    """Returns dict of error measures; o_* numpy float64 arrays of the same shape."""
+    o32 = np.asarray(o_f32_dev, dtype=np.float64)
+    ref = np.asarray(o_ref, dtype=np.float64)
+    max_abs = float(np.max(np.abs(o32 - ref))) if o32.size else 0.0
+    rel_l2 = float(np.linalg.norm(o32 - ref) / max(np.linalg.norm(ref), 1e-300)) if o32.size else 0.0
+    lse_d = np.asarray(lse_dev, dtype=np.float64)
+    lse_r = np.asarray(lse_ref, dtype=np.float64)
+    both_inf = np.isinf(lse_d) & np.isinf(lse_r)
+    lse_err = float(np.max(np.where(both_inf, 0.0, np.abs(lse_d - lse_r)))) if lse_d.size else 0.0
+    return {"max_abs": max_abs, "rel_l2": rel_l2, "lse_abs": lse_err}
+
+
+def bf16_is_rne_of_f32(o_bf16: torch.Tensor, o_f32: torch.Tensor) -> bool:
+    return torch.equal(o_f32.to(torch.bfloat16).view(torch.int16), o_bf16.view(torch.int16))
+
+
+def check_attention(errs, what=""):
+    assert errs["max_abs"] <= O_MAX_ABS, f"{what}: max abs {errs['max_abs']}"
+    assert errs["rel_l2"] <= O_REL_L2, f"{what}: rel L2 {errs['rel_l2']}"
+    assert errs["lse_abs"] <= LSE_ABS, f"{what}: lse err {errs['lse_abs']}"
+
+
+# ------------------------------------------------------------------ decode rows
+def logical_rows(X: torch.Tensor, page_table, b: int, g: int, token_ids: np.ndarray):
+    """Gather logical token rows (b, g, ids) of a contiguous or paged cache (any device)."""
+    ids = torch.from_numpy(np.asarray(token_ids, dtype=np.int64)).to(X.device)
+    if page_table is None:
+        return X[b, g, ids]
+    pages = page_table[b].long()[ids // 64]
+    return X[pages, g, ids % 64]
+
+
+def oracle_decode_row(w, inputs, b, g, kept_override=None):
+    """Oracle decode for row (b, g), gathering only the tokens it needs."""
+    G = w.G
+    lens = inputs["seq_lens"]
+    T_b = int(lens[b])
+    q_g = f64(inputs["q"][b, g * G:(g + 1) * G])
+    qi_g = f64(inputs["q_idx"][b, g * G:(g + 1) * G])
+    ki_g = f64(inputs["k_idx"][b, g, :T_b])
+    hw = f64(inputs["head_w"][g * G:(g + 1) * G])
+    S = O.decode_block_scores(qi_g, ki_g, T_b, hw, 1.0 / math.sqrt(w.r))
+    sel = O.select_decode(S, w.n_sink, w.n_local, w.p, w.k_max, w.k_min)
+    kept = sel.kept if kept_override is None else list(kept_override)
+    ids = O.kept_token_ids(kept, T_b)
+    K_tok = f64(logical_rows(inputs["K"], inputs.get("page_table"), b, g, ids))
+    V_tok = f64(logical_rows(inputs["V"], inputs.get("page_table"), b, g, ids))
+    o, lse = O.attend(q_g, K_tok, V_tok, 1.0 / math.sqrt(w.d))
+    return {"S": S, "sel": sel, "o": o, "lse": lse, "kept": kept}
+
+
+def compare_decode_rows(w, inputs, step, rows, p_override=None):
+    """Compare a finished DecodeStep with the oracle on the given (b, g) rows.
+
+    Returns a summary dict; raises AssertionError on any bar violation."""
+    G = w.G
+    kept = step.kept.cpu()
+    cnt = step.kept_count.cpu()
+    scores = step.scores.cpu()
+    o = step.o.cpu()
+    o32 = step.o_f32.cpu()
+    lse = step.lse.cpu()
+    assert bf16_is_rne_of_f32(o, o32), "bf16 output is not RNE(fp32 output)"
+    summary = {"rows": 0, "ties": 0, "max_abs": 0.0, "rel_l2": 0.0, "lse_abs": 0.0,
+               "score_rel": 0.0}
+    for (b, g) in rows:
+        ref = oracle_decode_row(w, inputs, b, g)
+        nb = len(ref["S"])
+        S_dev = scores[b, g, :nb].double().numpy()
+        if nb:
+            rel = np.max(np.abs(S_dev - ref["S"]) / np.maximum(1.0, np.abs(ref["S"])))
+            summary["score_rel"] = max(summary["score_rel"], float(rel))
+            assert rel <= SCORE_REL, f"row {(b, g)}: score rel err {rel}"
+        c = int(cnt[b, g])
+        kd = kept[b, g, :c].tolist()
+        assert all(x == -1 for x in kept[b, g, c:].tolist()), "padding is not -1"
+        verdict = selection_verdict(ref["sel"], kd, w.p)
+        assert not verdict.startswith("mismatch"), f"row {(b, g)}: {verdict}"
+        if verdict == "tie":
+            summary["ties"] += 1
+            ref = oracle_decode_row(w, inputs, b, g, kept_override=kd)
+        errs = attention_errors(o32[b, g * G:(g + 1) * G].double().numpy(), None,
+                                lse[b, g * G:(g + 1) * G].double().numpy(), ref["o"], ref["lse"])
+        check_attention(errs, f"row {(b, g)}")
+        for k_ in ("max_abs", "rel_l2", "lse_abs"):
+            summary[k_] = max(summary[k_], errs[k_])
+        summary["rows"] += 1
+    return summary
+
+
+# ------------------------------------------------------------------ prefill rows
+def oracle_prefill_rows(w, inputs, b, g, rows, kept_override=None):
+    G = w.G
+    T = w.T
+    q_g = f64(inputs["q"][b, g * G:(g + 1) * G, :T])
+    qi_g = f64(inputs["q_idx"][b, g * G:(g + 1) * G, :T])
+    ki_g = f64(inputs["k_idx"][b, g, :T])
+    K_g = f64(inputs["K"][b, g, :T])
+    V_g = f64(inputs["V"][b, g, :T])
+    hw = f64(inputs["head_w"][g * G:(g + 1) * G])
+    return O.prefill_rows(q_g, qi_g, ki_g, K_g, V_g, T, hw, 1.0 / math.sqrt(w.r),
+                          1.0 / math.sqrt(w.d), w.n_sink, w.n_local, w.p, w.k_max, w.k_min,
+                          rows=rows, kept_override=kept_override)
+
+
+def compare_prefill_rows(w, inputs, pf, b, g, rows):
+    G, T = w.G, w.T
+    kept = pf.kept.cpu()
+    cnt = pf.kept_count.cpu()
+    scores = pf.scores.cpu()
+    o = pf.o.cpu()
+    o32 = pf.o_f32.cpu()
+    lse = pf.lse.cpu()
+    summary = {"rows": 0, "ties": 0, "max_abs": 0.0, "rel_l2": 0.0, "lse_abs": 0.0,
+               "score_rel": 0.0}
+    refs = oracle_prefill_rows(w, inputs, b, g, rows)
+    override = {}
+    for i, ref in refs.items():
+        if i:
+            S_dev = scores[b, g, i, :i].double().numpy()
+            rel = np.max(np.abs(S_dev - ref["S"]) / np.maximum(1.0, np.abs(ref["S"])))
+            summary["score_rel"] = max(summary["score_rel"], float(rel))
+            assert rel <= SCORE_REL, f"prefill row {(b, g, i)}: score rel err {rel}"
+        c = int(cnt[b, g, i])
+        kd = kept[b, g, i, :c].tolist()
+        assert all(x == -1 for x in kept[b, g, i, c:].tolist()), "padding is not -1"
+        verdict = selection_verdict(ref["sel"], kd, w.p)
+        assert not verdict.startswith("mismatch"), f"prefill row {(b, g, i)}: {verdict}"
+        if verdict == "tie":
+            summary["ties"] += 1
+            override[i] = kd
+    if override:
+        refs.update(oracle_prefill_rows(w, inputs, b, g, list(override), kept_override=override))
+    for i, ref in refs.items():
+        q0, q1 = i * 64, min(i * 64 + 64, T)
+        o32_blk = o32[b, g * G:(g + 1) * G, q0:q1].double().numpy()
+        lse_blk = lse[b, g * G:(g + 1) * G, q0:q1].double().numpy()
+        errs = attention_errors(o32_blk, None, lse_blk, ref["o"], ref["lse"])
+        check_attention(errs, f"prefill row {(b, g, i)}")
+        for k_ in ("max_abs", "rel_l2", "lse_abs"):
+            summary[k_] = max(summary[k_], errs[k_])
+        summary["rows"] += 1
+    assert bf16_is_rne_of_f32(o[b, g * G:(g + 1) * G], o32[b, g * G:(g + 1) * G])
+    return summary
