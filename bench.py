@@ -1,0 +1,455 @@
+"""Benchmark: 128K-context batched decode + 64K block-sparse prefill on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole hot path: a decode step on the 128K workload
+(index scoring -> top-p selection -> split-K sparse attention) and a block-sparse
+causal prefill of the 64K workload (prefill scoring -> top-k selection -> sparse
+attention). Rank 0 prints one JSON line. Under torchrun each rank runs its own
+copy of the workload on its GPU (independent sequences, no data-path
+collective: weak scaling); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import block_sparse_long_06_b200 as bsa                      # noqa: E402
+from block_sparse_long_06_b200 import workloads as W         # noqa: E402
+
+METRIC = "decode tokens/s & achieved HBM GB/s at 128K ctx; sparse-prefill TFLOP/s"
+DECODE_WL = "decode_b32_h32_t128k_paged"
+PREFILL_WL = "prefill_b1_h32_t64k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "block_sparse_long_06_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key, files):
+    """Per-launch DRAM bytes from the committed ncu summary, if the kernel source
+    still matches the one the counters were taken on; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(kernel_key)
+    if not ent or ent.get("source_hash") != kernel_source_hash(files):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- byte / FLOP accounting
+def decode_bytes(w, kept_count, seq_lens):
+    """Algorithmic bytes of one decode step and of its attention call."""
+    B, Hq, Hkv, d, r = w.B, w.Hq, w.Hkv, w.d, w.r
+    kc = kept_count.to(torch.int64).cpu()
+    lens = seq_lens.to(torch.int64).cpu()
+    kv = int(kc.sum()) * 64 * d * 2 * 2                 # K and V of every kept block
+    idx = int(lens.sum()) * Hkv * r * 2                 # every index key
+    q = B * Hq * d * 2
+    q_idx = B * Hq * r * 2
+    o = B * Hq * d * 2 + B * Hq * 4                     # bf16 output + fp32 lse
+    pt = int(kc.sum()) * 4 if w.paged else 0            # page-table entries of kept blocks
+    attn = kv + q + o + pt
+    return {"step": kv + idx + q + q_idx + o + pt, "attention": attn, "index_keys": idx,
+            "kv": kv}
+
+
+def prefill_flops(w, kept_count):
+    kc = kept_count.to(torch.int64).cpu()
+    return float(kc.sum()) * w.G * 4 * 64 * 64 * w.d
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, world, rank, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    wd = W.WORKLOADS[DECODE_WL].with_(seed=rank)
+    wp = W.WORKLOADS[PREFILL_WL].with_(seed=rank)
+
+    xd = W.make_decode_inputs(wd, dev)
+    dprob = bsa.problem_for(wd, seq_lens=xd["seq_lens"], head_w=xd["head_w"])
+    dstep = bsa.DecodeStep(dprob, device=dev, keep_f32=False)
+    k_idx_c, K_c, V_c = bsa.caches_for(xd)
+
+    xp = W.make_prefill_inputs(wp, dev)
+    pprob = bsa.problem_for(wp, head_w=xp["head_w"])
+    pf = bsa.Prefill(pprob, device=dev, keep_f32=False)
+    pk_idx = bsa.contiguous_cache(xp["k_idx"])
+    pK = bsa.contiguous_cache(xp["K"])
+    pV = bsa.contiguous_cache(xp["V"])
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one_step(ev=None):
+        # decode on the 128K workload
+        if ev:
+            ev["d0"].record(stream)
+        bsa.bsa_score_blocks(dprob, xd["q_idx"], k_idx_c, dstep.scores, dstep.status)
+        bsa.bsa_select_top_p(dprob, dstep.scores, dstep.kept, dstep.kept_count, dstep.status)
+        if ev:
+            ev["a0"].record(stream)
+        bsa.bsa_decode(dprob, xd["q"], K_c, V_c, dstep.kept, dstep.kept_count, dstep.o,
+                       dstep.lse, None, dstep.workspace, dstep.status)
+        if ev:
+            ev["d1"].record(stream)
+        flush.zero_()                       # the prefill inputs fit in L2: flush before it
+        if ev:
+            ev["p0"].record(stream)
+        pf.select(xp["q_idx"], pk_idx)
+        if ev:
+            ev["p1"].record(stream)
+        pf.attend(xp["q"], pK, pV)
+        if ev:
+            ev["p2"].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    st = int(dstep.status.item()) | int(pf.status.item())
+    if st:
+        raise RuntimeError(f"device status {st:#x}")
+
+    names = ("d0", "a0", "d1", "p0", "p1", "p2")
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device() if world == 1 else local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for k in range(args.steps):
+            one_step(evs[k])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    dec_ms = [e["d0"].elapsed_time(e["d1"]) for e in evs]
+    att_ms = [e["a0"].elapsed_time(e["d1"]) for e in evs]
+    psel_ms = [e["p0"].elapsed_time(e["p1"]) for e in evs]
+    patt_ms = [e["p1"].elapsed_time(e["p2"]) for e in evs]
+    total_ms = t_start.elapsed_time(t_end)
+
+    dec_sum = max_over_ranks(sum(dec_ms), world)
+    step_ms = max_over_ranks(sum(d + ps + pa for d, ps, pa in zip(dec_ms, psel_ms, patt_ms)) /
+                             args.steps, world)
+    att_avg = max_over_ranks(sum(att_ms) / args.steps, world)
+    patt_avg = max_over_ranks(sum(patt_ms) / args.steps, world)
+    psel_avg = max_over_ranks(sum(psel_ms) / args.steps, world)
+    dec_avg = dec_sum / args.steps
+
+    by = decode_bytes(wd, dstep.kept_count, xd["seq_lens"])
+    flops = prefill_flops(wp, pf.kept_count)
+    tokens_per_s = world * wd.B * args.steps / (dec_sum / 1e3)
+    hbm = peaks["hbm_gbs"]
+    tflops_peak = peaks["bf16_tflops"]
+    attn_gbs = by["attention"] / (att_avg / 1e3) / 1e9
+    step_gbs = by["step"] / (dec_avg / 1e3) / 1e9
+    pf_tflops = flops / (patt_avg / 1e3) / 1e12
+
+    # end to end through the public API with host buffers (decode: the new query in,
+    # the attention output out, every step)
+    e2e = run_e2e(args, dprob, dstep, xd, k_idx_c, K_c, V_c, stream, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_decode(wd, xd, dstep, budget_s=args.cpu_budget)
+
+    clocks = clk.summary()
+    files = ["decode_attn.cu", "bsa_common.cuh", "bsa_internal.h"]
+    line = {
+        "metric": METRIC,
+        "value": tokens_per_s,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{DECODE_WL} + {PREFILL_WL}",
+            "decode": "B=32 Hq=32 Hkv=8 d=128 T=131072 paged KV (64-token pages), r=16, "
+                      "1 sink + 8 local, p=0.95, K_max=256",
+            "prefill": "B=1 Hq=32 Hkv=8 d=128 T=65536, diagonal + 1 sink + 2 local + top-64",
+            "l2": "decode inputs (18 GB) exceed L2; a 256 MB buffer is written before each prefill",
+            "parallelism": f"dp{world} (independent sequences per GPU)",
+        },
+        "decode": {"ms": dec_avg, "tokens_per_s": tokens_per_s, "hbm_gbs": step_gbs,
+                   "hbm_frac": step_gbs / hbm, "bytes_per_step": by["step"],
+                   "attention_ms": att_avg, "kept_blocks": int(dstep.kept_count.sum())},
+        "prefill": {"select_ms": psel_avg, "attention_ms": patt_avg, "tflops": pf_tflops,
+                    "tensor_frac": pf_tflops / tflops_peak, "kept_tile_flop": flops},
+        "roofline": {"bound": "hbm", "kernel": "bsa_decode (split-K attention + LSE merge)",
+                     "achieved": attn_gbs, "peak": hbm, "unit": "GB/s", "frac": attn_gbs / hbm,
+                     "traffic": ncu_traffic("decode_attn", files),
+                     "peak_source": f"{peak_src} hbm_gbs (burst copy)",
+                     "bytes_per_launch": by["attention"]},
+        "roofline_prefill": {"bound": "tensor", "kernel": "bsa_prefill (V->fp16 + attention)",
+                             "achieved": pf_tflops, "peak": tflops_peak, "unit": "TFLOP/s",
+                             "frac": pf_tflops / tflops_peak,
+                             "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "e2e": e2e,
+        "gpu_launches": args.steps * 8,
+        "clocks": clocks,
+        "total_ms_events": total_ms,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return line
+
+
+def run_e2e(args, dprob, dstep, xd, k_idx_c, K_c, V_c, stream, world):
+    q_h = xd["q"].cpu().pin_memory()
+    qi_h = xd["q_idx"].cpu().pin_memory()
+    o_h = torch.empty(dstep.o.shape, dtype=dstep.o.dtype).pin_memory()
+    lse_h = torch.empty(dstep.lse.shape, dtype=dstep.lse.dtype).pin_memory()
+    q_d = torch.empty_like(xd["q"])
+    qi_d = torch.empty_like(xd["q_idx"])
+
+    def step():
+        bsa.decode_step_host(dstep, q_h, qi_h, k_idx_c, K_c, V_c, o_h, lse_h, q_d, qi_d)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    B = dprob.B
+    return {"value": world * B * args.steps / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": q_h.numel() * 2 + qi_h.numel() * 2,
+            "d2h_bytes_per_step": o_h.numel() * 2 + lse_h.numel() * 4}
+
+
+# ---------------------------------------------------------------- oracle on the host
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline_decode(w, xd, dstep=None, budget_s=20.0, max_seqs=None):
+    """Time the fp64 oracle (as it stands) on a bounded sample of decode rows of the
+    workload: whole sequences (all kv heads) until ~budget_s of CPU work."""
+    from oracle import bsa_oracle as O
+    G, T = w.G, w.T
+    pt = xd.get("page_table")
+    done_seqs, t_total = 0, 0.0
+    b = 0
+    while b < w.B and (max_seqs is None or done_seqs < max_seqs):
+        # host copies of this sequence's inputs (not timed: a CPU program would hold them)
+        q = xd["q"][b].cpu()
+        qi = xd["q_idx"][b].cpu()
+        ki = xd["k_idx"][b].cpu()
+        if pt is None:
+            Kb, Vb = xd["K"][b].cpu(), xd["V"][b].cpu()
+            pages = None
+        else:
+            pages = pt[b].long()
+            Kb = xd["K"][pages].transpose(0, 1).reshape(w.Hkv, -1, w.d)[:, :T].cpu()
+            Vb = xd["V"][pages].transpose(0, 1).reshape(w.Hkv, -1, w.d)[:, :T].cpu()
+        hw = xd["head_w"].double().cpu().numpy()
+        t0 = time.perf_counter()
+        for g in range(w.Hkv):
+            S = O.decode_block_scores(qi[g * G:(g + 1) * G].double().numpy(),
+                                      ki[g, :T].double().numpy(), T, hw[g * G:(g + 1) * G],
+                                      1.0 / math.sqrt(w.r))
+            sel = O.select_decode(S, w.n_sink, w.n_local, w.p, w.k_max, w.k_min)
+            ids = O.kept_token_ids(sel.kept, T)
+            O.attend(q[g * G:(g + 1) * G].double().numpy(), Kb[g, ids].double().numpy(),
+                     Vb[g, ids].double().numpy(), 1.0 / math.sqrt(w.d))
+        t_total += time.perf_counter() - t0
+        done_seqs += 1
+        b += 1
+        if t_total >= budget_s:
+            break
+    return {"value": done_seqs / t_total, "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{done_seqs} of {w.B} sequences of {w.name} (all {w.Hkv} kv heads each: "
+                      f"score, select, attend in float64), {t_total:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    """The oracle on the host cores, same config / metric / unit, bounded per step."""
+    if rank != 0:
+        return None
+    wd = W.WORKLOADS[DECODE_WL]
+    if torch.cuda.is_available():
+        xd = W.make_decode_inputs(wd, "cuda")
+    else:
+        wd = wd.with_(B=2)
+        xd = W.make_decode_inputs(wd, "cpu")
+    per_step = []
+    for k in range(args.warmup + args.steps):
+        r = cpu_baseline_decode(wd, xd, budget_s=0.0, max_seqs=1)
+        if k >= args.warmup:
+            per_step.append(1.0 / r["value"])     # seconds for one sequence
+    sec = sum(per_step)
+    value = args.steps / sec
+    cpu = {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": f"one sequence (all {wd.Hkv} kv heads) of {DECODE_WL} per step"}
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": DECODE_WL, "parallelism": "host cores of rank 0"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    world, rank, local = dist_init()
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+    else:
+        line = run_ours(args, world, rank, local)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

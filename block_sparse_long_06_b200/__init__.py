@@ -299,3 +299,22 @@ def caches_for(inputs: dict):
         pt = inputs["page_table"]
         return k_idx, paged_cache(inputs["K"], pt), paged_cache(inputs["V"], pt)
     return k_idx, contiguous_cache(inputs["K"]), contiguous_cache(inputs["V"])
+
+
+def decode_step_host(step: DecodeStep, q_host, q_idx_host, k_idx: Cache, k: Cache, v: Cache,
+                     o_host, lse_host, q_dev=None, q_idx_dev=None, stream=None):
+    """One decode step from host buffers: copy the new query (q, q_idx; pinned host
+    tensors) to the device, run score -> select -> attend, copy o and lse back into
+    the pinned host tensors, and wait for them. The KV and index-key caches stay
+    resident on the device."""
+    stream = torch.cuda.current_stream() if stream is None else stream
+    q_dev = torch.empty(q_host.shape, dtype=q_host.dtype, device="cuda") if q_dev is None else q_dev
+    q_idx_dev = (torch.empty(q_idx_host.shape, dtype=q_idx_host.dtype, device="cuda")
+                 if q_idx_dev is None else q_idx_dev)
+    with torch.cuda.stream(stream):
+        q_dev.copy_(q_host, non_blocking=True)
+        q_idx_dev.copy_(q_idx_host, non_blocking=True)
+        step.run(q_dev, q_idx_dev, k_idx, k, v, stream)
+        o_host.copy_(step.o, non_blocking=True)
+        lse_host.copy_(step.lse, non_blocking=True)
+    stream.synchronize()

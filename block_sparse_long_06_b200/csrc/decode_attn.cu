@@ -65,8 +65,10 @@ BSA_DEVFN int seq_len(const DecodeArgs& a, int b) {
   return Tb < 0 ? 0 : (Tb > a.T ? a.T : Tb);
 }
 
-// Row (in rows of width d) of the first token of block `blk` of (b, g); -1 if invalid.
-BSA_DEVFN int64_t tile_row(const CacheView& c, int b, int g, int blk, int d) {
+// Row (in rows of width d) of the first token of block `blk` of (b, g); -1 if the
+// page id is invalid or the `rows` existing tokens of the block leave the extent.
+// (TMA fills rows of a box beyond the tensor with zeros; those tokens are masked.)
+BSA_DEVFN int64_t tile_row(const CacheView& c, int b, int g, int blk, int rows, int d) {
   int64_t phys = blk;
   if (c.page_table != nullptr) {
     phys = c.page_table[static_cast<int64_t>(b) * c.pt_stride + blk];
@@ -74,7 +76,7 @@ BSA_DEVFN int64_t tile_row(const CacheView& c, int b, int g, int blk, int d) {
   }
   const int64_t off = static_cast<int64_t>(b) * c.seq_stride + phys * c.block_stride +
                       static_cast<int64_t>(g) * c.head_stride;
-  if (off < 0 || off + static_cast<int64_t>(kBlock) * d > c.extent) return -1;
+  if (off < 0 || off + static_cast<int64_t>(rows) * d > c.extent) return -1;
   return off / d;
 }
 
@@ -118,7 +120,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = row / a.Hkv, g = row % a.Hkv;
         const int cnt = min(a.kept_count[row], a.max_kept);
         const int e0 = sp * a.split_len, e1 = min(cnt, e0 + a.split_len);
-        const int nb = (seq_len(a, b) + kBlock - 1) / kBlock;
+        const int Tb = seq_len(a, b);
+        const int nb = (Tb + kBlock - 1) / kBlock;
         for (int e = e0; e < e1; ++e, ++it) {
           const int s = it % S;
           if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
@@ -129,8 +132,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int blk = a.kept[static_cast<int64_t>(row) * a.max_kept + e];
           int64_t rk = -1, rv = -1;
           if (blk >= 0 && blk < nb) {
-            rk = tile_row(a.k, b, g, blk, D);
-            rv = tile_row(a.v, b, g, blk, D);
+            const int rows = min(kBlock, Tb - blk * kBlock);
+            rk = tile_row(a.k, b, g, blk, rows, D);
+            rv = tile_row(a.v, b, g, blk, rows, D);
             if (rk < 0 || rv < 0) report(a.status, BSA_DEV_BAD_PAGE);
           } else {
             report(a.status, BSA_DEV_BAD_KEPT);

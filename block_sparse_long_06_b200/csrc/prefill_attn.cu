@@ -36,7 +36,7 @@ struct PCfg {
                                kStages * 4 + 1024;
 };
 
-BSA_DEVFN int64_t prow(const CacheView& c, int b, int g, int blk, int d) {
+BSA_DEVFN int64_t prow(const CacheView& c, int b, int g, int blk, int rows, int d) {
   int64_t phys = blk;
   if (c.page_table != nullptr) {
     phys = c.page_table[static_cast<int64_t>(b) * c.pt_stride + blk];
@@ -44,7 +44,7 @@ BSA_DEVFN int64_t prow(const CacheView& c, int b, int g, int blk, int d) {
   }
   const int64_t off = static_cast<int64_t>(b) * c.seq_stride + phys * c.block_stride +
                       static_cast<int64_t>(g) * c.head_stride;
-  if (off < 0 || off + static_cast<int64_t>(kBlock) * d > c.extent) return -1;
+  if (off < 0 || off + static_cast<int64_t>(rows) * d > c.extent) return -1;
   return off / d;
 }
 
@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         const int blk = klist[e];
         int64_t rk = -1;
         if (blk >= 0 && blk <= i) {
-          rk = prow(a.k, b, g, blk, D);
+          rk = prow(a.k, b, g, blk, min(kBlock, a.T - blk * kBlock), D);
           if (rk < 0) report(a.status, BSA_DEV_BAD_PAGE);
         } else {
           report(a.status, BSA_DEV_BAD_KEPT);

@@ -49,8 +49,9 @@ BSA_DEVFN ItemGeom item_geom(const ScoreDecodeArgs& a, int64_t item) {
   return it;
 }
 
-// Element offset of block `blk` of (b, g); false when the page id or extent check fails.
-BSA_DEVFN bool block_offset(const CacheView& c, int b, int g, int blk, int64_t& off) {
+// Element offset of block `blk` of (b, g); false when the page id or extent check
+// fails for the `rows` tokens of the block that exist.
+BSA_DEVFN bool block_offset(const CacheView& c, int b, int g, int blk, int rows, int64_t& off) {
   int64_t phys = blk;
   if (c.page_table != nullptr) {
     phys = c.page_table[static_cast<int64_t>(b) * c.pt_stride + blk];
@@ -58,7 +59,12 @@ BSA_DEVFN bool block_offset(const CacheView& c, int b, int g, int blk, int64_t& 
   }
   off = static_cast<int64_t>(b) * c.seq_stride + phys * c.block_stride +
         static_cast<int64_t>(g) * c.head_stride;
-  return off >= 0 && off + kBlock * kR <= c.extent;
+  return off >= 0 && off + static_cast<int64_t>(rows) * kR <= c.extent;
+}
+
+BSA_DEVFN int rows_of(const ItemGeom& it, int j) {
+  const int r = it.Tb - j * kBlock;
+  return r < kBlock ? r : kBlock;
 }
 
 template <int NT>
@@ -89,18 +95,22 @@ __global__ void __launch_bounds__(kWarps * 32) score_decode_kernel(const ScoreDe
     const ItemGeom it = item_geom(a, item);
     uint32_t bytes = 0;
     int64_t offs[kStageBlocks];
-    bool ok[kStageBlocks];
+    uint32_t nbytes[kStageBlocks];
 #pragma unroll
     for (int q = 0; q < kStageBlocks; ++q) {
       const int j = it.j0 + q;
-      ok[q] = (j < it.nb_row) && block_offset(a.kidx, it.b, it.g, j, offs[q]);
-      if (ok[q]) bytes += kBlockBytes;
+      nbytes[q] = 0;
+      if (j < it.nb_row) {
+        const int rows = rows_of(it, j);   // a partial last block copies only its tokens
+        if (block_offset(a.kidx, it.b, it.g, j, rows, offs[q])) nbytes[q] = rows * kR * 2;
+      }
+      bytes += nbytes[q];
     }
     mbar_arrive_expect_tx(&bars[s], bytes);
 #pragma unroll
     for (int q = 0; q < kStageBlocks; ++q)
-      if (ok[q])
-        bulk_g2s(ring + s * kStageBytes + q * kBlockBytes, kbase + offs[q] * 2, kBlockBytes,
+      if (nbytes[q])
+        bulk_g2s(ring + s * kStageBytes + q * kBlockBytes, kbase + offs[q] * 2, nbytes[q],
                  &bars[s]);
   };
 
@@ -151,7 +161,7 @@ __global__ void __launch_bounds__(kWarps * 32) score_decode_kernel(const ScoreDe
         continue;
       }
       int64_t off_unused;
-      if (!block_offset(a.kidx, it.b, it.g, j, off_unused)) {
+      if (!block_offset(a.kidx, it.b, it.g, j, rows_of(it, j), off_unused)) {
         if (lane == 0) {
           out[j] = -INFINITY;
           report(a.status, BSA_DEV_BAD_PAGE);
