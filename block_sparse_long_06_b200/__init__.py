@@ -27,7 +27,9 @@ OP_SCORE, OP_SELECT, OP_DECODE, OP_PREFILL = 0, 1, 2, 3
 BLOCK = 64
 
 EXPORTED = ["bsa_max_kept", "bsa_workspace_size", "bsa_score_blocks", "bsa_select_top_p",
-            "bsa_decode", "bsa_prefill", "bsa_status_string", "bsa_last_cuda_error"]
+            "bsa_decode", "bsa_prefill", "bsa_status_string", "bsa_last_cuda_error",
+            "bsa_decode_noalloc"]
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class BsaError(RuntimeError):
@@ -76,6 +78,8 @@ def load_library(path: str = LIB_PATH):
         f = getattr(lib, name)
         f.argtypes = [P, vp, CCache, CCache, vp, vp, vp, vp, vp, vp, sz, vp, vp]
         f.restype = ctypes.c_int
+    lib.bsa_decode_noalloc.argtypes = [P, vp, CCache, CCache, vp, vp, vp, vp, vp, vp, vp]
+    lib.bsa_decode_noalloc.restype = ctypes.c_int
     lib.bsa_status_string.argtypes = [ctypes.c_int]
     lib.bsa_status_string.restype = ctypes.c_char_p
     lib.bsa_last_cuda_error.argtypes = []
@@ -212,6 +216,17 @@ def bsa_prefill(prob: Problem, q, k: Cache, v: Cache, kept, kept_count, o, lse, 
                                       _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                       _ptr(dev_status), _stream(stream)),
            "bsa_prefill")
+
+
+def bsa_decode_noalloc(prob: Problem, q, k: Cache, v: Cache, kept, kept_count, o, lse, o_f32,
+                       dev_status=None, stream=None):
+    """bsa_decode without a workspace argument, for callers that cannot allocate device
+    memory: the split-K scratch lives in the library's fixed 8 MiB device array. Calls
+    that overlap on the GPU share that array and must be serialised by the caller."""
+    _check(load_library().bsa_decode_noalloc(ctypes.byref(prob.c()), _ptr(q), k.c(), v.c(),
+                                             _ptr(kept), _ptr(kept_count), _ptr(o), _ptr(lse),
+                                             _ptr(o_f32), _ptr(dev_status), _stream(stream)),
+           "bsa_decode_noalloc")
 
 
 def bsa_status_string(status: int) -> str:

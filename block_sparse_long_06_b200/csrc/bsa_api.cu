@@ -151,6 +151,10 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 }  // namespace
 
+namespace bsa {
+bsa_status_t record_cuda_error(cudaError_t e) { return cuda_fail(e); }
+}  // namespace bsa
+
 extern "C" {
 
 int32_t bsa_max_kept(const bsa_problem_t* p) {

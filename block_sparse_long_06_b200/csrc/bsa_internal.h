@@ -91,6 +91,9 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tq, const CU
                            const CUtensorMap& tv16, int num_sms, cudaStream_t s);
 cudaError_t launch_v_to_f16(const PrefillArgs& a, cudaStream_t s);
 
+// Records a CUDA error for bsa_last_cuda_error() and returns BSA_ERR_CUDA.
+bsa_status_t record_cuda_error(cudaError_t e);
+
 // Decode split-K geometry chosen on the host from the worst-case kept count.
 void decode_split_plan(int rows, int max_kept, int num_sms, int* splits, int* split_len);
 

@@ -150,6 +150,27 @@ bsa_status_t bsa_prefill(const bsa_problem_t* prob, const void* q, bsa_cache_t k
                          float* o_f32, void* workspace, size_t workspace_bytes,
                          int32_t* dev_status, void* stream);
 
+/* Size of the fixed device scratch array used by bsa_decode_noalloc (8 MiB). */
+#define BSA_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* Decode attention without a caller-provided workspace, for callers that cannot
+ * allocate device memory (a host framework that owns every allocation, a plugin
+ * with a memory budget fixed at start-up, a path where cudaMalloc would stall the
+ * device). It has no counterpart on the pages: it is bsa_decode with its split-K
+ * scratch placed in a file-scope device array of BSA_NOALLOC_SCRATCH_BYTES that
+ * every device loading this library reserves until the process exits.
+ * Arguments and outputs are those of bsa_decode minus the workspace. Returns
+ * BSA_ERR_WORKSPACE, launching nothing, when the problem needs more scratch than
+ * BSA_NOALLOC_SCRATCH_BYTES (bsa_workspace_size(BSA_OP_DECODE) tells how much).
+ * The first call on a device looks up the array's address (cudaGetSymbolAddress)
+ * with that device current; make it before any stream capture. All calls on a
+ * device share the array: calls whose work overlaps on the GPU race and must be
+ * serialised by the caller. Allocates and frees nothing. */
+bsa_status_t bsa_decode_noalloc(const bsa_problem_t* prob, const void* q, bsa_cache_t k,
+                                bsa_cache_t v, const int32_t* kept, const int32_t* kept_count,
+                                void* o, float* lse, float* o_f32, int32_t* dev_status,
+                                void* stream);
+
 /* Static description of a status code. */
 const char* bsa_status_string(bsa_status_t status);
 
