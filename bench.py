@@ -84,10 +84,13 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.dev)],
+                 "-lms", "20", "-i", str(self.dev)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 5.0:   # sampling has started
+                time.sleep(0.01)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -182,20 +185,23 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
-    wd = W.WORKLOADS[DECODE_WL].with_(seed=rank)
-    wp = W.WORKLOADS[PREFILL_WL].with_(seed=rank)
+    do_dec = args.phase in ("both", "decode")
+    do_pf = args.phase in ("both", "prefill")
+    wd = W.WORKLOADS[args.decode_workload].with_(seed=rank)
+    wp = W.WORKLOADS[args.prefill_workload].with_(seed=rank)
 
     xd = W.make_decode_inputs(wd, dev)
     dprob = bsa.problem_for(wd, seq_lens=xd["seq_lens"], head_w=xd["head_w"])
     dstep = bsa.DecodeStep(dprob, device=dev, keep_f32=False)
     k_idx_c, K_c, V_c = bsa.caches_for(xd)
 
-    xp = W.make_prefill_inputs(wp, dev)
-    pprob = bsa.problem_for(wp, head_w=xp["head_w"])
-    pf = bsa.Prefill(pprob, device=dev, keep_f32=False)
-    pk_idx = bsa.contiguous_cache(xp["k_idx"])
-    pK = bsa.contiguous_cache(xp["K"])
-    pV = bsa.contiguous_cache(xp["V"])
+    if do_pf:
+        xp = W.make_prefill_inputs(wp, dev)
+        pprob = bsa.problem_for(wp, head_w=xp["head_w"])
+        pf = bsa.Prefill(pprob, device=dev, keep_f32=False)
+        pk_idx = bsa.contiguous_cache(xp["k_idx"])
+        pK = bsa.contiguous_cache(xp["K"])
+        pV = bsa.contiguous_cache(xp["V"])
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -203,28 +209,33 @@ def run_ours(args, world, rank, local):
         # decode on the 128K workload
         if ev:
             ev["d0"].record(stream)
-        bsa.bsa_score_blocks(dprob, xd["q_idx"], k_idx_c, dstep.scores, dstep.status)
-        bsa.bsa_select_top_p(dprob, dstep.scores, dstep.kept, dstep.kept_count, dstep.status)
+        if do_dec:
+            bsa.bsa_score_blocks(dprob, xd["q_idx"], k_idx_c, dstep.scores, dstep.status)
+            bsa.bsa_select_top_p(dprob, dstep.scores, dstep.kept, dstep.kept_count, dstep.status)
         if ev:
             ev["a0"].record(stream)
-        bsa.bsa_decode(dprob, xd["q"], K_c, V_c, dstep.kept, dstep.kept_count, dstep.o,
-                       dstep.lse, None, dstep.workspace, dstep.status)
+        if do_dec:
+            bsa.bsa_decode(dprob, xd["q"], K_c, V_c, dstep.kept, dstep.kept_count, dstep.o,
+                           dstep.lse, None, dstep.workspace, dstep.status)
         if ev:
             ev["d1"].record(stream)
-        flush.zero_()                       # the prefill inputs fit in L2: flush before it
+        if do_pf:
+            flush.zero_()                   # the prefill inputs fit in L2: flush before it
         if ev:
             ev["p0"].record(stream)
-        pf.select(xp["q_idx"], pk_idx)
+        if do_pf:
+            pf.select(xp["q_idx"], pk_idx)
         if ev:
             ev["p1"].record(stream)
-        pf.attend(xp["q"], pK, pV)
+        if do_pf:
+            pf.attend(xp["q"], pK, pV)
         if ev:
             ev["p2"].record(stream)
 
     for _ in range(args.warmup):
         one_step()
     torch.cuda.synchronize()
-    st = int(dstep.status.item()) | int(pf.status.item())
+    st = int(dstep.status.item()) | (int(pf.status.item()) if do_pf else 0)
     if st:
         raise RuntimeError(f"device status {st:#x}")
 
@@ -256,7 +267,11 @@ def run_ours(args, world, rank, local):
     dec_avg = dec_sum / args.steps
 
     by = decode_bytes(wd, dstep.kept_count, xd["seq_lens"])
-    flops = prefill_flops(wp, pf.kept_count)
+    flops = prefill_flops(wp, pf.kept_count) if do_pf else 0.0
+    dec_sum = max(dec_sum, 1e-9)
+    patt_avg = max(patt_avg, 1e-9)
+    att_avg = max(att_avg, 1e-9)
+    dec_avg = max(dec_avg, 1e-9)
     tokens_per_s = world * wd.B * args.steps / (dec_sum / 1e3)
     hbm = peaks["hbm_gbs"]
     tflops_peak = peaks["bf16_tflops"]
@@ -266,7 +281,8 @@ def run_ours(args, world, rank, local):
 
     # end to end through the public API with host buffers (decode: the new query in,
     # the attention output out, every step)
-    e2e = run_e2e(args, dprob, dstep, xd, k_idx_c, K_c, V_c, stream, world)
+    e2e = (None if args.no_e2e or not do_dec else
+           run_e2e(args, dprob, dstep, xd, k_idx_c, K_c, V_c, stream, world))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -288,7 +304,8 @@ def run_ours(args, world, rank, local):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": f"{DECODE_WL} + {PREFILL_WL}",
+            "workload": f"{wd.name} + {wp.name}" if args.phase == "both" else
+                        (wd.name if do_dec else wp.name),
             "decode": "B=32 Hq=32 Hkv=8 d=128 T=131072 paged KV (64-token pages), r=16, "
                       "1 sink + 8 local, p=0.95, K_max=256",
             "prefill": "B=1 Hq=32 Hkv=8 d=128 T=65536, diagonal + 1 sink + 2 local + top-64",
@@ -310,7 +327,7 @@ def run_ours(args, world, rank, local):
                              "frac": pf_tflops / tflops_peak,
                              "peak_source": f"{peak_src} bf16_tflops (burst)"},
         "e2e": e2e,
-        "gpu_launches": args.steps * 8,
+        "gpu_launches": args.steps * (4 * do_dec + 4 * do_pf),
         "clocks": clocks,
         "total_ms_events": total_ms,
     }
@@ -431,11 +448,17 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--phase", choices=["both", "decode", "prefill"], default="both")
+    ap.add_argument("--decode-workload", default=DECODE_WL, choices=sorted(
+        k for k, v in W.WORKLOADS.items() if v.phase == "decode"))
+    ap.add_argument("--prefill-workload", default=PREFILL_WL, choices=sorted(
+        k for k, v in W.WORKLOADS.items() if v.phase == "prefill"))
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -181,7 +181,7 @@ bsa_status_t bsa_workspace_size(const bsa_problem_t* p, int32_t op, size_t* byte
     case BSA_OP_PREFILL: {
       if (p->phase != BSA_PHASE_PREFILL) return BSA_ERR_INVALID_ARG;
       const int64_t Tpad = static_cast<int64_t>(nblocks(p->T)) * 64;
-      *bytes = align256(static_cast<size_t>(p->B) * p->Hkv * Tpad * p->d * 2);
+      *bytes = align256(static_cast<size_t>(p->B) * p->Hkv * Tpad * p->d * 2) + 256;
       return BSA_OK;
     }
     default:
@@ -213,7 +213,8 @@ bsa_status_t bsa_score_blocks(const bsa_problem_t* p, const void* q_idx, bsa_cac
     a.G = G;
     a.T = p->T;
     a.nb_max = nblocks(p->T);
-    a.chunks_per_row = (a.nb_max + 1) / 2;  // two blocks per stage
+    const int cb = bsa::score_decode_chunk_blocks();
+    a.chunks_per_row = (a.nb_max + cb - 1) / cb;
     a.total_items = static_cast<int64_t>(p->B) * p->Hkv * a.chunks_per_row;
     a.idx_scale = idx_scale_of(p);
     e = bsa::launch_score_decode(a, num_sms, s);
@@ -326,7 +327,8 @@ bsa_status_t bsa_prefill(const bsa_problem_t* p, const void* q, bsa_cache_t k, b
   if ((st = check_cache(v, p, p->d, false)) != BSA_OK) return st;
   const int nqb = nblocks(p->T);
   const int64_t Tpad = static_cast<int64_t>(nqb) * 64;
-  const size_t need = align256(static_cast<size_t>(p->B) * p->Hkv * Tpad * p->d * 2);
+  const size_t v16_bytes = align256(static_cast<size_t>(p->B) * p->Hkv * Tpad * p->d * 2);
+  const size_t need = v16_bytes + 256;
   if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return BSA_ERR_WORKSPACE;
   const int64_t qrows = static_cast<int64_t>(p->B) * p->Hq * p->T;
@@ -360,7 +362,8 @@ bsa_status_t bsa_prefill(const bsa_problem_t* p, const void* q, bsa_cache_t k, b
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = bsa::launch_v_to_f16(a, s);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = bsa::launch_prefill(a, tq, tk, tv, num_sms_current(), s);
+  int* unit_counter = reinterpret_cast<int*>(static_cast<char*>(workspace) + v16_bytes);
+  e = bsa::launch_prefill_tc(a, tq, tk, tv, unit_counter, num_sms_current(), s);
   return e == cudaSuccess ? BSA_OK : cuda_fail(e);
 }
 

@@ -87,9 +87,13 @@ cudaError_t launch_score_prefill(const ScorePrefillArgs& a, int num_sms, cudaStr
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                           int num_units, int num_sms, cudaStream_t s);
-cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
-                           const CUtensorMap& tv16, int num_sms, cudaStream_t s);
 cudaError_t launch_v_to_f16(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv16, int* unit_counter, int num_sms,
+                              cudaStream_t s);
+
+// Blocks per work item of the decode scorer (items are (row, chunk) pairs).
+int score_decode_chunk_blocks();
 
 // Records a CUDA error for bsa_last_cuda_error() and returns BSA_ERR_CUDA.
 bsa_status_t record_cuda_error(cudaError_t e);

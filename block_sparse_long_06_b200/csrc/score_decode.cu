@@ -6,47 +6,51 @@
 //  RTPurbo, Methodology §2: r = 16 index keys; block aggregate = max).
 //
 // Design (HBM-bound stream of 32 bytes per token):
-//  * warp-private rings of 1-D bulk copies (cp.async.bulk + mbarrier): each stage
-//    holds kStageBlocks blocks of 64 tokens x 16 bf16 = 2 KB; a warp owns a
-//    contiguous range of (row, chunk) items, so its reads are sequential;
-//  * the 16-dim dot products run on the tensor cores: mma.m16n8k16 with the
-//    tokens as M (16 per tile), the group's heads as N (8 per tile, zero padded),
-//    K = r = 16. The K dimension is relabelled so that each lane's fragment is one
-//    8-byte run of a token (lane t holds dims 4t..4t+3), which makes the shared
-//    memory reads conflict-free 64-bit loads; the query fragment uses the same
-//    relabelling, so every dot product is unchanged;
+//  * persistent CTAs, each owning a contiguous range of items; an item is a chunk
+//    of kChunk consecutive blocks of one row (16 KB of index keys). One producer
+//    lane computes the item's geometry once, publishes it in shared memory and
+//    streams the chunk into a ring of stages with 1-D bulk copies (one copy per
+//    chunk when the blocks are contiguous, one per block otherwise), completion
+//    counted on per-stage "full" mbarriers;
+//  * consumer warp w scores block w of every chunk. The 16-dim dot products run
+//    on mma.m16n8k16 with tokens as M (16 per tile), the group's heads as N (8 per
+//    tile, zero padded) and K = r = 16. The K dimension is relabelled so that each
+//    lane's fragment is one 8-byte run of a token (lane t holds dims 4t..4t+3):
+//    shared-memory reads are conflict-free 64-bit loads, and the query fragment
+//    uses the same relabelling, so every dot product is unchanged;
 //  * epilogue in fp32: ReLU, head weights, head sum with two shuffles (each lane
-//    pair exchanges the half it does not keep), running max, then a 4-shuffle
-//    warp max per block.
+//    pair exchanges the half it does not keep), running max, a 4-shuffle warp max
+//    per block, then the stage is released through its "empty" mbarrier.
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
 
 namespace bsa {
 namespace {
 
-constexpr int kWarps = 4;          // warps per CTA
-constexpr int kStages = 4;         // ring depth per warp
-constexpr int kStageBlocks = 2;    // 64-token blocks per stage
-constexpr int kBlockBytes = kBlock * kR * 2;                 // 2048
-constexpr int kStageBytes = kStageBlocks * kBlockBytes;      // 4096
-constexpr int kCtasPerSm = 3;
+constexpr int kConsumers = 8;                              // consumer warps = blocks per chunk
+constexpr int kChunk = kConsumers;                         // blocks per item / stage
+constexpr int kStages = 6;
+constexpr int kBlockBytes = kBlock * kR * 2;               // 2048
+constexpr int kStageBytes = kChunk * kBlockBytes;          // 16 KB
+constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kCtasPerSm = 2;
 
-struct ItemGeom {
-  int row, b, g, j0, nb_row, Tb;
+struct StageInfo {
+  int row;        // b * Hkv + g
+  int j0;         // first block of the chunk
+  int Tb;         // tokens of sequence b
+  uint32_t ok;    // bit q: block j0 + q was copied
 };
 
-BSA_DEVFN ItemGeom item_geom(const ScoreDecodeArgs& a, int64_t item) {
-  ItemGeom it;
-  it.row = static_cast<int>(item / a.chunks_per_row);
-  const int chunk = static_cast<int>(item % a.chunks_per_row);
-  it.b = it.row / a.Hkv;
-  it.g = it.row % a.Hkv;
-  it.j0 = chunk * kStageBlocks;
-  int Tb = a.seq_lens ? a.seq_lens[it.b] : a.T;
-  Tb = Tb < 0 ? 0 : (Tb > a.T ? a.T : Tb);
-  it.Tb = Tb;
-  it.nb_row = (Tb + kBlock - 1) / kBlock;
-  return it;
+struct ScoreSmem {
+  static constexpr int kRing = kStages * kStageBytes;
+  static constexpr int kInfo = kStages * static_cast<int>(sizeof(StageInfo));
+  static constexpr int kTotal = kRing + kInfo + 2 * kStages * 8 + 128;
+};
+
+BSA_DEVFN int clamp_len(const ScoreDecodeArgs& a, int b) {
+  int Tb = a.seq_lens ? a.seq_lens[b] : a.T;
+  return Tb < 0 ? 0 : (Tb > a.T ? a.T : Tb);
 }
 
 // Element offset of block `blk` of (b, g); false when the page id or extent check
@@ -62,73 +66,114 @@ BSA_DEVFN bool block_offset(const CacheView& c, int b, int g, int blk, int rows,
   return off >= 0 && off + static_cast<int64_t>(rows) * kR <= c.extent;
 }
 
-BSA_DEVFN int rows_of(const ItemGeom& it, int j) {
-  const int r = it.Tb - j * kBlock;
-  return r < kBlock ? r : kBlock;
-}
-
 template <int NT>
-__global__ void __launch_bounds__(kWarps * 32) score_decode_kernel(const ScoreDecodeArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  unsigned char* ring = smem + warp * (kStages * kStageBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kStages * kStageBytes) + warp * kStages;
+__global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecodeArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
+  unsigned char* ring = smem;
+  StageInfo* info = reinterpret_cast<StageInfo*>(smem + ScoreSmem::kRing);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ScoreSmem::kRing + ScoreSmem::kInfo);
+  uint64_t* empty = full + kStages;
 
-  if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers);
+    }
     fence_mbar_init();
   }
-  __syncwarp();
+  __syncthreads();
 
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-  const int64_t per = (a.total_items + nwarps - 1) / nwarps;
-  const int64_t it_begin = gw * per;
-  const int64_t it_end = min(a.total_items, it_begin + per);
-  const int64_t n_items = it_end > it_begin ? it_end - it_begin : 0;
-  const char* kbase = static_cast<const char*>(a.kidx.base);
+  const int64_t per = (a.total_items + gridDim.x - 1) / gridDim.x;
+  const int64_t it0 = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t it1 = min(a.total_items, it0 + per);
+  const int n_items = it1 > it0 ? static_cast<int>(it1 - it0) : 0;
 
-  // lane 0 issues the copies of one item into one stage
-  auto issue = [&](int64_t item, int s) {
-    if (lane != 0) return;
-    const ItemGeom it = item_geom(a, item);
-    uint32_t bytes = 0;
-    int64_t offs[kStageBlocks];
-    uint32_t nbytes[kStageBlocks];
-#pragma unroll
-    for (int q = 0; q < kStageBlocks; ++q) {
-      const int j = it.j0 + q;
-      nbytes[q] = 0;
-      if (j < it.nb_row) {
-        const int rows = rows_of(it, j);   // a partial last block copies only its tokens
-        if (block_offset(a.kidx, it.b, it.g, j, rows, offs[q])) nbytes[q] = rows * kR * 2;
+  if (warp == kConsumers) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      const char* kbase = static_cast<const char*>(a.kidx.base);
+      const bool contiguous = a.kidx.page_table == nullptr && a.kidx.block_stride == kBlock * kR;
+      // walk the item range incrementally: (row, j0) without a division per item
+      int row = static_cast<int>(it0 / a.chunks_per_row);
+      int j0 = static_cast<int>(it0 - static_cast<int64_t>(row) * a.chunks_per_row) * kChunk;
+      int b = row / a.Hkv, g = row - b * a.Hkv;
+      int Tb = clamp_len(a, b);
+      for (int k = 0; k < n_items; ++k) {
+        const int s = k % kStages;
+        if (!mbar_wait(&empty[s], ((k / kStages) & 1) ^ 1)) {
+          report(a.status, BSA_DEV_TIMEOUT);
+          break;
+        }
+        const int nb_row = (Tb + kBlock - 1) / kBlock;
+        const int nblk = max(0, min(kChunk, nb_row - j0));      // blocks of the chunk that exist
+        unsigned char* dst = ring + s * kStageBytes;
+        uint32_t ok = 0, bytes = 0;
+        if (contiguous && nblk > 0) {
+          // the chunk's blocks are adjacent: one range check, one copy
+          const int rows = min(nblk * kBlock, Tb - j0 * kBlock);
+          int64_t off;
+          if (block_offset(a.kidx, b, g, j0, rows, off)) {
+            ok = (1u << nblk) - 1u;
+            bytes = rows * kR * 2;
+          }
+          info[s] = StageInfo{row, j0, Tb, ok};
+          mbar_arrive_expect_tx(&full[s], bytes);
+          if (ok) bulk_g2s(dst, kbase + off * 2, bytes, &full[s]);
+        } else {
+          int64_t offs[kChunk];
+          int rows_q[kChunk];
+          for (int q = 0; q < nblk; ++q) {
+            rows_q[q] = min(kBlock, Tb - (j0 + q) * kBlock);
+            if (block_offset(a.kidx, b, g, j0 + q, rows_q[q], offs[q])) {
+              ok |= 1u << q;
+              bytes += rows_q[q] * kR * 2;
+            }
+          }
+          info[s] = StageInfo{row, j0, Tb, ok};
+          mbar_arrive_expect_tx(&full[s], bytes);
+          for (int q = 0; q < nblk; ++q)
+            if (ok & (1u << q))
+              bulk_g2s(dst + q * kBlockBytes, kbase + offs[q] * 2, rows_q[q] * kR * 2, &full[s]);
+        }
+        // next item
+        j0 += kChunk;
+        if (j0 >= a.chunks_per_row * kChunk) {
+          j0 = 0;
+          ++row;
+          if (++g == a.Hkv) {
+            g = 0;
+            ++b;
+            if (b < a.B) Tb = clamp_len(a, b);
+          }
+        }
       }
-      bytes += nbytes[q];
+      // let the consumers release what was issued before the CTA can exit (bounded)
+      for (int k = max(0, n_items - kStages); k < n_items; ++k)
+        mbar_wait(&empty[k % kStages], (k / kStages) & 1, 200000000ull);
     }
-    mbar_arrive_expect_tx(&bars[s], bytes);
-#pragma unroll
-    for (int q = 0; q < kStageBlocks; ++q)
-      if (nbytes[q])
-        bulk_g2s(ring + s * kStageBytes + q * kBlockBytes, kbase + offs[q] * 2, nbytes[q],
-                 &bars[s]);
-  };
+    return;
+  }
 
-  const int pre = static_cast<int>(n_items < kStages ? n_items : kStages);
-  for (int s = 0; s < pre; ++s) issue(it_begin + s, s);
-
+  // ------------------------------------------------------------------ consumers
+  const int gid = lane >> 2, tig = lane & 3;
   int cur_row = -1;
   uint32_t bq[NT][2];
   float w0[NT], w1[NT];
-  bool timed_out = false;
-
-  for (int64_t k = 0; k < n_items; ++k) {
-    const int s = static_cast<int>(k % kStages);
-    const uint32_t parity = static_cast<uint32_t>((k / kStages) & 1);
-    const ItemGeom it = item_geom(a, it_begin + k);
-    if (it.row != cur_row) {
-      cur_row = it.row;
-      // query fragment: lane (gid, tig) holds head 8*nt + gid, dims 4*tig .. 4*tig+3
+  for (int k = 0; k < n_items; ++k) {
+    const int s = k % kStages;
+    if (!mbar_wait(&full[s], (k / kStages) & 1)) {
+      if (lane == 0) report(a.status, BSA_DEV_TIMEOUT);
+      break;
+    }
+    const StageInfo in = info[s];
+    const int j = in.j0 + warp;
+    if (in.row != cur_row) {
+      cur_row = in.row;
+      const int b = in.row / a.Hkv, g = in.row - b * a.Hkv;
+      const float dflt = 1.0f / static_cast<float>(a.G);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int hl = nt * 8 + gid;
@@ -136,91 +181,67 @@ __global__ void __launch_bounds__(kWarps * 32) score_decode_kernel(const ScoreDe
         if (hl < a.G) {
           const uint2 v = *reinterpret_cast<const uint2*>(
               static_cast<const char*>(a.q_idx) +
-              ((static_cast<int64_t>(it.b) * a.Hq + it.g * a.G + hl) * kR + 4 * tig) * 2);
+              ((static_cast<int64_t>(b) * a.Hq + g * a.G + hl) * kR + 4 * tig) * 2);
           bq[nt][0] = v.x;
           bq[nt][1] = v.y;
         }
         const int h0 = nt * 8 + 2 * tig, h1 = h0 + 1;
-        const float dflt = 1.0f / static_cast<float>(a.G);
-        w0[nt] = h0 < a.G ? (a.head_w ? a.head_w[it.g * a.G + h0] : dflt) : 0.f;
-        w1[nt] = h1 < a.G ? (a.head_w ? a.head_w[it.g * a.G + h1] : dflt) : 0.f;
+        w0[nt] = h0 < a.G ? (a.head_w ? a.head_w[g * a.G + h0] : dflt) : 0.f;
+        w1[nt] = h1 < a.G ? (a.head_w ? a.head_w[g * a.G + h1] : dflt) : 0.f;
       }
     }
-    if (!mbar_wait(&bars[s], parity)) {
-      timed_out = true;
-      break;
-    }
-    const unsigned char* st = ring + s * kStageBytes;
-    float* out = a.scores + static_cast<int64_t>(it.row) * a.nb_max;
-#pragma unroll
-    for (int q = 0; q < kStageBlocks; ++q) {
-      const int j = it.j0 + q;
-      if (j >= a.nb_max) break;
-      if (j >= it.nb_row) {
-        if (lane == 0) out[j] = -INFINITY;
-        continue;
-      }
-      int64_t off_unused;
-      if (!block_offset(a.kidx, it.b, it.g, j, rows_of(it, j), off_unused)) {
+    if (j < a.nb_max) {
+      float* out = a.scores + static_cast<int64_t>(in.row) * a.nb_max + j;
+      const int valid = in.Tb - j * kBlock;  // tokens of this block that exist
+      if (valid <= 0) {
+        if (lane == 0) *out = -INFINITY;
+      } else if (!(in.ok & (1u << warp))) {
         if (lane == 0) {
-          out[j] = -INFINITY;
+          *out = -INFINITY;
           report(a.status, BSA_DEV_BAD_PAGE);
         }
-        continue;
-      }
-      const unsigned char* blk = st + q * kBlockBytes;
-      const int valid = it.Tb - j * kBlock;  // tokens of this block that exist (>= 1)
-      float mx = 0.f;
-#pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        const int r0 = mt * 16 + gid, r1 = r0 + 8;
-        const uint2 x0 = *reinterpret_cast<const uint2*>(blk + r0 * 32 + tig * 8);
-        const uint2 x1 = *reinterpret_cast<const uint2*>(blk + r1 * 32 + tig * 8);
-        const uint32_t af[4] = {x0.x, x1.x, x0.y, x1.y};
-        float vr0 = 0.f, vr1 = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          float c[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_bf16(c, af, bq[nt][0], bq[nt][1]);
-          vr0 = fmaf(w0[nt], fmaxf(c[0], 0.f), vr0);
-          vr0 = fmaf(w1[nt], fmaxf(c[1], 0.f), vr0);
-          vr1 = fmaf(w0[nt], fmaxf(c[2], 0.f), vr1);
-          vr1 = fmaf(w1[nt], fmaxf(c[3], 0.f), vr1);
-        }
-        // head sum over the 4 lanes of a row group: even lanes keep token r0,
-        // odd lanes token r1
+      } else {
+        const unsigned char* blk = ring + s * kStageBytes + warp * kBlockBytes;
+        float mx = 0.f;
         const bool odd = tig & 1;
-        const float send = odd ? vr0 : vr1;
-        float keep = odd ? vr1 : vr0;
-        keep += __shfl_xor_sync(0xffffffffu, send, 1);
-        keep += __shfl_xor_sync(0xffffffffu, keep, 2);
-        const int tok = odd ? r1 : r0;
-        if (tok < valid) mx = fmaxf(mx, keep);
-      }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      if (lane == 0) {
-        const float sc = a.idx_scale * mx;
-        out[j] = sc;
-        if (!isfinite(sc)) report(a.status, BSA_DEV_NONFINITE);
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          const int r0 = mt * 16 + gid, r1 = r0 + 8;
+          const uint2 x0 = *reinterpret_cast<const uint2*>(blk + r0 * 32 + tig * 8);
+          const uint2 x1 = *reinterpret_cast<const uint2*>(blk + r1 * 32 + tig * 8);
+          const uint32_t af[4] = {x0.x, x1.x, x0.y, x1.y};
+          float vr0 = 0.f, vr1 = 0.f;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_bf16(c, af, bq[nt][0], bq[nt][1]);
+            vr0 = fmaf(w0[nt], fmaxf(c[0], 0.f), vr0);
+            vr0 = fmaf(w1[nt], fmaxf(c[1], 0.f), vr0);
+            vr1 = fmaf(w0[nt], fmaxf(c[2], 0.f), vr1);
+            vr1 = fmaf(w1[nt], fmaxf(c[3], 0.f), vr1);
+          }
+          // head sum over the 4 lanes of a row group: even lanes keep token r0,
+          // odd lanes token r1
+          const float send = odd ? vr0 : vr1;
+          float keep = odd ? vr1 : vr0;
+          keep += __shfl_xor_sync(0xffffffffu, send, 1);
+          keep += __shfl_xor_sync(0xffffffffu, keep, 2);
+          const int tok = odd ? r1 : r0;
+          if (tok < valid) mx = fmaxf(mx, keep);
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        if (lane == 0) {
+          const float sc = a.idx_scale * mx;
+          *out = sc;
+          if (!isfinite(sc)) report(a.status, BSA_DEV_NONFINITE);
+        }
       }
     }
     __syncwarp();
-    if (k + kStages < n_items) {
-      fence_proxy_async_smem();
-      issue(it_begin + k + kStages, s);
-    }
-  }
-
-  if (timed_out) {
-    if (lane == 0) report(a.status, BSA_DEV_TIMEOUT);
-    // let copies still in flight land before the CTA exits (bounded)
-    for (int64_t k = 0; k < n_items && k < kStages; ++k) {
-      const int64_t kk = n_items - 1 - k;
-      mbar_wait(&bars[kk % kStages], static_cast<uint32_t>((kk / kStages) & 1), 100000000ull);
-    }
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
 }
 
@@ -228,17 +249,16 @@ __global__ void __launch_bounds__(kWarps * 32) score_decode_kernel(const ScoreDe
 
 cudaError_t launch_score_decode(const ScoreDecodeArgs& a, int num_sms, cudaStream_t s) {
   if (a.total_items <= 0) return cudaSuccess;
-  const size_t smem = kWarps * kStages * kStageBytes + kWarps * kStages * sizeof(uint64_t);
-  int64_t warps_needed = a.total_items;
-  int64_t ctas = (warps_needed + kWarps - 1) / kWarps;
-  const int64_t cap = static_cast<int64_t>(num_sms) * kCtasPerSm;
-  if (ctas > cap) ctas = cap;
+  const int smem = ScoreSmem::kTotal;
+  int64_t ctas = static_cast<int64_t>(num_sms) * kCtasPerSm;
+  if (ctas > a.total_items) ctas = a.total_items;
   auto kern = (a.G > 8) ? score_decode_kernel<2> : score_decode_kernel<1>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>(ctas), kWarps * 32, smem, s>>>(a);
+  kern<<<static_cast<unsigned>(ctas), kThreads, smem, s>>>(a);
   return cudaGetLastError();
 }
+
+int score_decode_chunk_blocks() { return kChunk; }
 
 }  // namespace bsa
