@@ -181,6 +181,16 @@ def prefill_flops(w, kept_count):
 
 
 # ---------------------------------------------------------------- our arm
+def describe(w) -> str:
+    """One-line description of a workload, from its fields."""
+    kv = "paged KV (64-token pages)" if w.paged else "contiguous KV"
+    base = f"B={w.B} Hq={w.Hq} Hkv={w.Hkv} d={w.d} T={w.T} {kv}, r={w.r}"
+    if w.phase == "decode":
+        return f"{base}, {w.n_sink} sink + {w.n_local} local, p={w.p}, K_max={w.k_max}"
+    sel = f"top-{w.k_max}" if w.p >= 1.0 else f"p={w.p}, K_max={w.k_max}"
+    return f"{base}, diagonal + {w.n_sink} sink + {w.n_local} local + {sel}"
+
+
 def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -190,11 +200,11 @@ def run_ours(args, world, rank, local):
     wd = W.WORKLOADS[args.decode_workload].with_(seed=rank)
     wp = W.WORKLOADS[args.prefill_workload].with_(seed=rank)
 
-    xd = W.make_decode_inputs(wd, dev)
-    dprob = bsa.problem_for(wd, seq_lens=xd["seq_lens"], head_w=xd["head_w"])
-    dstep = bsa.DecodeStep(dprob, device=dev, keep_f32=False)
-    k_idx_c, K_c, V_c = bsa.caches_for(xd)
-
+    if do_dec:
+        xd = W.make_decode_inputs(wd, dev)
+        dprob = bsa.problem_for(wd, seq_lens=xd["seq_lens"], head_w=xd["head_w"])
+        dstep = bsa.DecodeStep(dprob, device=dev, keep_f32=False)
+        k_idx_c, K_c, V_c = bsa.caches_for(xd)
     if do_pf:
         xp = W.make_prefill_inputs(wp, dev)
         pprob = bsa.problem_for(wp, head_w=xp["head_w"])
@@ -206,7 +216,6 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     def one_step(ev=None):
-        # decode on the 128K workload
         if ev:
             ev["d0"].record(stream)
         if do_dec:
@@ -235,7 +244,7 @@ def run_ours(args, world, rank, local):
     for _ in range(args.warmup):
         one_step()
     torch.cuda.synchronize()
-    st = int(dstep.status.item()) | (int(pf.status.item()) if do_pf else 0)
+    st = (int(dstep.status.item()) if do_dec else 0) | (int(pf.status.item()) if do_pf else 0)
     if st:
         raise RuntimeError(f"device status {st:#x}")
 
@@ -258,6 +267,7 @@ def run_ours(args, world, rank, local):
     patt_ms = [e["p1"].elapsed_time(e["p2"]) for e in evs]
     total_ms = t_start.elapsed_time(t_end)
 
+    # every rank takes the same collective steps, whatever the phase
     dec_sum = max_over_ranks(sum(dec_ms), world)
     step_ms = max_over_ranks(sum(d + ps + pa for d, ps, pa in zip(dec_ms, psel_ms, patt_ms)) /
                              args.steps, world)
@@ -265,19 +275,40 @@ def run_ours(args, world, rank, local):
     patt_avg = max_over_ranks(sum(patt_ms) / args.steps, world)
     psel_avg = max_over_ranks(sum(psel_ms) / args.steps, world)
     dec_avg = dec_sum / args.steps
-
-    by = decode_bytes(wd, dstep.kept_count, xd["seq_lens"])
-    flops = prefill_flops(wp, pf.kept_count) if do_pf else 0.0
-    dec_sum = max(dec_sum, 1e-9)
-    patt_avg = max(patt_avg, 1e-9)
-    att_avg = max(att_avg, 1e-9)
-    dec_avg = max(dec_avg, 1e-9)
-    tokens_per_s = world * wd.B * args.steps / (dec_sum / 1e3)
     hbm = peaks["hbm_gbs"]
     tflops_peak = peaks["bf16_tflops"]
-    attn_gbs = by["attention"] / (att_avg / 1e3) / 1e9
-    step_gbs = by["step"] / (dec_avg / 1e3) / 1e9
-    pf_tflops = flops / (patt_avg / 1e3) / 1e12
+
+    dec = pre = None
+    roof_dec = roof_pf = None
+    if do_dec:
+        by = decode_bytes(wd, dstep.kept_count, xd["seq_lens"])
+        dec_sum, att_avg, dec_avg = max(dec_sum, 1e-9), max(att_avg, 1e-9), max(dec_avg, 1e-9)
+        tokens_per_s = world * wd.B * args.steps / (dec_sum / 1e3)
+        attn_gbs = by["attention"] / (att_avg / 1e3) / 1e9
+        step_gbs = by["step"] / (dec_avg / 1e3) / 1e9
+        dec = {"ms": dec_avg, "tokens_per_s": tokens_per_s, "hbm_gbs": step_gbs,
+               "hbm_frac": step_gbs / hbm, "bytes_per_step": by["step"],
+               "attention_ms": att_avg, "kept_blocks": int(dstep.kept_count.sum())}
+        files = ["decode_attn.cu", "bsa_common.cuh", "bsa_internal.h"]
+        roof_dec = {"bound": "hbm", "kernel": "bsa_decode (split-K attention + LSE merge)",
+                    "achieved": attn_gbs, "peak": hbm, "unit": "GB/s", "frac": attn_gbs / hbm,
+                    "traffic": ncu_traffic("decode_attn", files),
+                    "peak_source": f"{peak_src} hbm_gbs (burst copy)",
+                    "bytes_per_launch": by["attention"]}
+    if do_pf:
+        flops = prefill_flops(wp, pf.kept_count)
+        patt_avg = max(patt_avg, 1e-9)
+        pf_tflops = world * flops / (patt_avg / 1e3) / 1e12
+        pre = {"select_ms": psel_avg, "attention_ms": patt_avg, "tflops": pf_tflops,
+               "tensor_frac": pf_tflops / world / tflops_peak, "kept_tile_flop": flops}
+        files = ["prefill_tc.cu", "prefill_attn.cu", "tcgen05.cuh", "bsa_common.cuh",
+                 "bsa_internal.h"]
+        roof_pf = {"bound": "tensor", "kernel": "bsa_prefill (V->fp16 + attention)",
+                   "achieved": pf_tflops / world, "peak": tflops_peak, "unit": "TFLOP/s",
+                   "frac": pf_tflops / world / tflops_peak,
+                   "traffic": ncu_traffic("prefill_tc", files),
+                   "peak_source": f"{peak_src} bf16_tflops (burst)",
+                   "flop_per_launch": flops}
 
     # end to end through the public API with host buffers (decode: the new query in,
     # the attention output out, every step)
@@ -285,15 +316,28 @@ def run_ours(args, world, rank, local):
            run_e2e(args, dprob, dstep, xd, k_idx_c, K_c, V_c, stream, world))
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and do_dec:
         cpu = cpu_baseline_decode(wd, xd, dstep, budget_s=args.cpu_budget)
 
     clocks = clk.summary()
-    files = ["decode_attn.cu", "bsa_common.cuh", "bsa_internal.h"]
+    config = {"workload": " + ".join(w.name for w, on in ((wd, do_dec), (wp, do_pf)) if on)}
+    if do_dec:
+        config["decode"] = describe(wd)
+    if do_pf:
+        config["prefill"] = describe(wp)
+    config["l2"] = ("decode inputs exceed L2; a 256 MB buffer is written before each prefill")
+    config["parallelism"] = f"dp{world} (independent sequences per GPU)"
+    # kernels per step: decode = scorer, selection, split-K attention, LSE merge;
+    # prefill = scorer, selection, V->fp16, attention
+    launches = args.steps * (4 * do_dec + 4 * do_pf)
+    if do_dec:
+        value, unit = dec["tokens_per_s"], "tokens/s"
+    else:
+        value, unit = pre["tflops"], "TFLOP/s"
     line = {
         "metric": METRIC,
-        "value": tokens_per_s,
-        "unit": "tokens/s",
+        "value": value,
+        "unit": unit,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -303,34 +347,17 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": f"{wd.name} + {wp.name}" if args.phase == "both" else
-                        (wd.name if do_dec else wp.name),
-            "decode": "B=32 Hq=32 Hkv=8 d=128 T=131072 paged KV (64-token pages), r=16, "
-                      "1 sink + 8 local, p=0.95, K_max=256",
-            "prefill": "B=1 Hq=32 Hkv=8 d=128 T=65536, diagonal + 1 sink + 2 local + top-64",
-            "l2": "decode inputs (18 GB) exceed L2; a 256 MB buffer is written before each prefill",
-            "parallelism": f"dp{world} (independent sequences per GPU)",
-        },
-        "decode": {"ms": dec_avg, "tokens_per_s": tokens_per_s, "hbm_gbs": step_gbs,
-                   "hbm_frac": step_gbs / hbm, "bytes_per_step": by["step"],
-                   "attention_ms": att_avg, "kept_blocks": int(dstep.kept_count.sum())},
-        "prefill": {"select_ms": psel_avg, "attention_ms": patt_avg, "tflops": pf_tflops,
-                    "tensor_frac": pf_tflops / tflops_peak, "kept_tile_flop": flops},
-        "roofline": {"bound": "hbm", "kernel": "bsa_decode (split-K attention + LSE merge)",
-                     "achieved": attn_gbs, "peak": hbm, "unit": "GB/s", "frac": attn_gbs / hbm,
-                     "traffic": ncu_traffic("decode_attn", files),
-                     "peak_source": f"{peak_src} hbm_gbs (burst copy)",
-                     "bytes_per_launch": by["attention"]},
-        "roofline_prefill": {"bound": "tensor", "kernel": "bsa_prefill (V->fp16 + attention)",
-                             "achieved": pf_tflops, "peak": tflops_peak, "unit": "TFLOP/s",
-                             "frac": pf_tflops / tflops_peak,
-                             "peak_source": f"{peak_src} bf16_tflops (burst)"},
-        "e2e": e2e,
-        "gpu_launches": args.steps * (4 * do_dec + 4 * do_pf),
-        "clocks": clocks,
-        "total_ms_events": total_ms,
+        "config": config,
     }
+    if dec is not None:
+        line["decode"] = dec
+    if pre is not None:
+        line["prefill"] = pre
+    line["roofline"] = roof_dec if roof_dec is not None else roof_pf
+    if roof_dec is not None and roof_pf is not None:
+        line["roofline_prefill"] = roof_pf
+    line.update({"e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+                 "total_ms_events": total_ms})
     if cpu is not None:
         line["cpu_baseline"] = cpu
     return line

@@ -70,6 +70,30 @@ BSA_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 200
   }
 }
 
+// As mbar_try_wait, but the thread is suspended (it takes no issue slots) until
+// the phase completes or about `hint_ns` have passed.
+BSA_DEVFN bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait that sleeps instead of spinning: for waits that are often long,
+// where spinning warps would take issue slots from the warps doing the work.
+BSA_DEVFN bool mbar_wait_sleep(uint64_t* bar, uint32_t parity,
+                               uint64_t limit_ns = 2000000000ull) {
+  if (mbar_try_wait_suspend(bar, parity, 100000u)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_suspend(bar, parity, 100000u)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // Order this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (bulk copy / TMA) accesses of the same buffer.
 BSA_DEVFN void fence_proxy_async_smem() {

@@ -11,30 +11,34 @@
 //    two 128-row Q tiles (two heads each). Persistent CTAs (one per SM) take units
 //    from a global counter in (b, g)-major, heavy-first order, so all SMs share the
 //    K/V of one kv head through L2 at a time;
-//  * kept key blocks are processed in pairs: a pair is a 128-key tile, so every
-//    MMA has N = 128 (a lone last block uses N = 64);
-//  * warp 0 (one lane) loads Q once per unit and the K tiles (bf16) of each pair
-//    into a K ring, and publishes each pair's block ids and mask modes in a small
-//    shared-memory ring; warp 2 (one lane) loads the V tiles (fp16) into a V ring.
-//    All loads are TMA with 128-byte swizzle;
-//  * warp 1 (one lane) issues the MMAs. S_t = Q_t K^T (bf16, M = 128, K = d) goes to
-//    tensor memory; O_t += P_t V (fp16, P read from tensor memory, N = d). Per pair
-//    k the order is S_0(k), P_1(k-1).V, S_1(k), P_0(k).V, so each tile's softmax
-//    runs while the tensor core works for the other tile. S_t(k) overwrites P_t(k-1)
-//    and therefore waits for the P.V of tile t on pair k-1;
-//  * warps 4-7 and 8-11 are the softmax warpgroups of tile 0 and tile 1 (a thread
-//    per row = tensor-memory lane). A thread loads its S row once (128 fp32), masks
-//    the causal diagonal block, takes the row max with three-input max, computes P
-//    with packed two-wide fp32 arithmetic and writes it as fp16 over the S columns
-//    it has consumed. 3/8 of the exponentials run as a cubic polynomial on the FMA
-//    pipes (exp2_poly below) instead of the MUFU unit, the co-bottleneck of
-//    attention at d = 128. The running max only moves (and O is rescaled in tensor
-//    memory) when it grows by more than 8 (log2), so P <= 256 fits fp16 and the
+//  * a step is one kept key block (64 keys) for both tiles. Warp 0 (one lane)
+//    loads Q once per unit and, per step, the K block (bf16) and the V block (fp16)
+//    into one stage of a K/V ring (TMA, 128-byte swizzle);
+//  * one MMA-issuing thread per tile (warps 1 and 2): a single thread can issue a
+//    tcgen05.mma only every ~50 cycles and a commit costs about as much, so one
+//    issuer for both tiles would leave the tensor core idle. Tile t's issuer runs
+//    S_t(j) = Q_t K_j^T (bf16, M = 128, N = 64, K = d) into one of the tile's two S
+//    buffers in tensor memory and O_t += P_t(j) V_j (fp16, P read from tensor
+//    memory over the S columns, N = d), in the order P_t(j).V, S_t(j+2): the score
+//    MMAs run two steps ahead, so the softmax of a tile goes from one step to the
+//    next without waiting for the tensor core. An S buffer is reused once the
+//    P.V that read it has completed; a K/V stage is released by the P.V of every
+//    tile;
+//  * warps 4-11 and 12-19 are the softmax warps of tile 0 and tile 1, 16 rows each
+//    (tensor-memory lane quarter = warp % 4). They read the step's block id from
+//    the kept list and validate it themselves, so the only per-step wait is for S.
+//    A thread holds 2 rows x 16 columns of S, masks the causal diagonal block (and
+//    blocks that failed validation), takes the row max (three-input max, then 2
+//    shuffles), computes P with packed two-wide fp32 arithmetic and writes it as
+//    fp16 over the S columns. 3/8 of the exponentials run as a cubic polynomial on
+//    the FMA pipes (exp2_poly below) instead of the MUFU unit. The running max only
+//    moves (and O is rescaled in tensor memory, after the previous P.V has
+//    completed) when it grows by more than 8 (log2), so P <= 256 fits fp16 and the
 //    rescale is rare; the final normalisation uses the same max, so it is exact;
 //  * epilogue: O / l from tensor memory straight to global memory (bf16, and fp32
 //    when requested), LSE in natural log.
-// Tensor memory: 512 columns: S/P of tile 0 at 0, of tile 1 at 128; O of tile 0 at
-// 256, of tile 1 at 384. Every wait is bounded; on a timeout the kernel sets
+// Tensor memory: 512 columns: O of tile t at 128 t; S/P buffer b of tile t at
+// 256 + 128 t + 64 b. Every wait is bounded; on a timeout the kernel sets
 // BSA_DEV_TIMEOUT, drains, frees its tensor memory and returns.
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
@@ -43,23 +47,23 @@
 namespace bsa {
 namespace {
 
-constexpr int kThreads = 384;
-constexpr int kWarpLoadK = 0, kWarpMma = 1, kWarpLoadV = 2, kWarpSm0 = 4;
+constexpr int kThreads = 640;
+constexpr int kWarpLoad = 0, kWarpMma0 = 1, kWarpSm0 = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kPI = 8;          // depth of the pair-info ring
-constexpr int kPolyPairs = 6;   // per 16 packed pairs of a 32-column chunk: computed by polynomial
+constexpr int kMaxStages = 8;
+constexpr int kPolyGroups = 3;  // of every 8 column groups of a row: exponentials by polynomial
 
 template <int D>
 struct Cfg {
-  static constexpr int kHalves = D / 64;          // 64-dim slabs of 128 rows x 128 B
-  static constexpr int kSlab = 128 * 128;
+  static constexpr int kHalves = D / 64;          // 64-dim slabs (rows of 128 B)
+  static constexpr int kSlab = 128 * 128;         // one slab of a 128-row Q tile
   static constexpr int kTile = kHalves * kSlab;   // 128 rows x D
-  static constexpr int kSK = D == 128 ? 3 : 4;    // K stages
-  static constexpr int kSV = D == 128 ? 2 : 4;    // V stages
+  static constexpr int kBlk = kHalves * 8192;     // one key block: 64 rows x D
+  static constexpr int kStage = 2 * kBlk;         // K block, then V block
+  static constexpr int kStages = D == 128 ? 5 : 8;
   static constexpr int kKsteps = D / 16;
-  static constexpr int kOffK = 2 * kTile;
-  static constexpr int kOffV = kOffK + kSK * kTile;
-  static constexpr int kOffBar = kOffV + kSV * kTile;
+  static constexpr int kOffKV = 2 * kTile;
+  static constexpr int kOffBar = kOffKV + kStages * kStage;
 };
 
 struct UnitInfo {
@@ -69,12 +73,11 @@ struct UnitInfo {
 struct Bars {
   uint64_t info_full[2], info_empty[2];
   uint64_t q_full, q_empty;
-  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
-  uint64_t pi_full[kPI], pi_empty[kPI];
-  uint64_t s_full[2], p_ready[2], o_done[2], o_free[2];
-  uint64_t mma_done;
+  uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
+  uint64_t s_full[2][2], p_ready[2][2], pv_done[2][2];   // [tile][S buffer]
+  uint64_t o_free[2];
+  uint64_t mma_done[2];
   UnitInfo info[2];
-  int4 pinfo[kPI];   // blk0, blk1, nb, mode0 | mode1 << 8   (mode: 0 visible, 1 diagonal, 2 masked)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -83,6 +86,7 @@ template <int D>
 constexpr int smem_bytes() {
   return Cfg<D>::kOffBar + static_cast<int>(sizeof(Bars)) + 1024;
 }
+static_assert(smem_bytes<128>() <= 232448, "shared memory");
 
 BSA_DEVFN bool aborted(Bars* b) { return *reinterpret_cast<volatile int*>(&b->abort_flag) != 0; }
 BSA_DEVFN void set_abort(Bars* b, int32_t* status) {
@@ -130,7 +134,7 @@ BSA_DEVFN int row_head(const PrefillArgs& a, int hq, int t, int r) {
 // (Polling from every lane only adds shared-memory traffic.)
 BSA_DEVFN bool warp_wait(uint64_t* bar, uint32_t parity) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity);
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_sleep(bar, parity);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
@@ -138,17 +142,6 @@ BSA_DEVFN float max3(float x, float y, float z) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(x), "f"(y), "f"(z));
   return r;
-}
-
-// Masks the 64 scores of one key block held in two 32-column chunks: columns past
-// `lim` (the last visible key offset; -1 hides the whole block) become -inf.
-BSA_DEVFN void mask_block(uint32_t (&c0)[32], uint32_t (&c1)[32], int lim) {
-  const uint32_t ninf = 0xff800000u;
-#pragma unroll
-  for (int x = 0; x < 32; ++x) {
-    if (x > lim) c0[x] = ninf;
-    if (x + 32 > lim) c1[x] = ninf;
-  }
 }
 
 // 2^x on the FMA pipes, for x <= 8 (two lanes at once). Split x = n + f with n the
@@ -173,6 +166,15 @@ BSA_DEVFN float2 exp2_poly(float2 x) {
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(r.y) << 23)));
 }
 
+
+
+// Mask mode of a kept block: 0 visible, 1 the causal diagonal, 2 failed validation
+// (the loader then loads the diagonal block in its place).
+BSA_DEVFN int mode_of(const PrefillArgs& a, const UnitInfo& U, int blk) {
+  if (krow_of(a.k, a, U.b, U.g, blk, U.i) < 0) return 2;
+  return blk == U.i ? 1 : 0;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tmq,
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmv, int* unit_counter,
                       const int num_units) {
   using C = Cfg<D>;
-  constexpr int SK = C::kSK, SV = C::kSV;
+  constexpr int NS = C::kStages;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -191,29 +193,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->info_full[x], 1);
-      mbar_init(&bars->info_empty[x], 1 + 1 + 8);   // MMA lane, V loader, every softmax warp
-      mbar_init(&bars->s_full[x], 1);
-      mbar_init(&bars->p_ready[x], 4);
-      mbar_init(&bars->o_done[x], 1);
-      mbar_init(&bars->o_free[x], 4);
+      mbar_init(&bars->info_empty[x], 2 + 16);    // both issuers, every softmax warp
+      for (int y = 0; y < 2; ++y) {
+        mbar_init(&bars->s_full[x][y], 1);
+        mbar_init(&bars->p_ready[x][y], 8);       // the 8 softmax warps of a tile
+        mbar_init(&bars->pv_done[x][y], 1);
+      }
+      mbar_init(&bars->o_free[x], 8);
+      mbar_init(&bars->mma_done[x], 1);
     }
-    for (int s = 0; s < 4; ++s) {
-      mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->k_empty[s], 1);
-      mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->v_empty[s], 1);
-    }
-    for (int s = 0; s < kPI; ++s) {
-      mbar_init(&bars->pi_full[s], 1);
-      mbar_init(&bars->pi_empty[s], 1 + 1 + 4 * ntiles);  // MMA lane, V loader, active softmax warps
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], ntiles);      // the P.V of every tile
     }
     mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
-    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->q_empty, ntiles);            // the last score MMAs of every tile
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpMma) {
+  if (warp == kWarpMma0) {
     tc::tmem_alloc(&bars->tmem_base, kTmemCols);
     tc::tmem_relinquish();
   }
@@ -222,11 +220,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == kWarpLoadK) {
-    // ---------------------------------------------------------- Q / K / pair info
+  if (warp == kWarpLoad) {
+    // -------------------------------------------------------------- Q / K / V
     if (lane == 0) {
       prefetch_tensormap(&tmq);
       prefetch_tensormap(&tmk);
+      prefetch_tensormap(&tmv);
       uint32_t un = 0, kc = 0;
       bool ok = true;
       while (ok) {
@@ -252,92 +251,52 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_2d(smem + t * C::kTile + x * C::kSlab + hh * 8192, &tmq, x * 64, qr,
                           &bars->q_full);
           }
-        const int npairs = (U.cnt + 1) / 2;
-        for (int pp = 0; pp < npairs; ++pp, ++kc) {
-          const int nb = (2 * pp + 1 < U.cnt) ? 2 : 1;
-          int blk[2] = {-1, -1}, mode[2] = {2, 2};
-          int64_t rk[2] = {0, 0};
-          for (int q = 0; q < nb; ++q) {
-            blk[q] = klist[2 * pp + q];
-            rk[q] = krow_of(a.k, a, U.b, U.g, blk[q], U.i);
-            if (rk[q] < 0) {
-              report(a.status, blk[q] < 0 || blk[q] > U.i ? BSA_DEV_BAD_KEPT : BSA_DEV_BAD_PAGE);
-              blk[q] = U.i;   // load the always-valid diagonal block; its columns are masked
-              rk[q] = krow_of(a.k, a, U.b, U.g, blk[q], U.i);
-              if (rk[q] < 0) rk[q] = 0;
-              mode[q] = 2;
-            } else {
-              mode[q] = blk[q] == U.i ? 1 : 0;
-            }
+        const int n = U.cnt > 0 ? U.cnt : 1;
+        const int32_t vrow0 = static_cast<int32_t>((static_cast<int64_t>(U.b) * a.Hkv + U.g) * a.Tpad);
+        for (int jj = 0; jj < n; ++jj, ++kc) {
+          int blk = U.i;
+          int64_t rk = -1;
+          if (jj < U.cnt) {
+            blk = klist[jj];
+            rk = krow_of(a.k, a, U.b, U.g, blk, U.i);
+            if (rk < 0)
+              report(a.status, blk < 0 || blk > U.i ? BSA_DEV_BAD_KEPT : BSA_DEV_BAD_PAGE);
           }
-          const int pi = kc % kPI;
-          if (!mbar_wait(&bars->pi_empty[pi], ((kc / kPI) & 1) ^ 1)) { ok = false; break; }
-          bars->pinfo[pi] = make_int4(blk[0], blk[1], nb, mode[0] | (mode[1] << 8));
-          mbar_arrive(&bars->pi_full[pi]);
-          const int s = kc % SK;
-          if (!mbar_wait(&bars->k_empty[s], ((kc / SK) & 1) ^ 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars->k_full[s], nb * C::kHalves * 8192);
-          unsigned char* kst = smem + C::kOffK + s * C::kTile;
-          for (int q = 0; q < nb; ++q)
-            for (int x = 0; x < C::kHalves; ++x)
-              tma_load_2d(kst + x * C::kSlab + q * 8192, &tmk, x * 64, static_cast<int32_t>(rk[q]),
-                          &bars->k_full[s]);
+          if (rk < 0) {
+            blk = U.i;   // load the always-valid diagonal block; its columns are masked
+            rk = krow_of(a.k, a, U.b, U.g, blk, U.i);
+            if (rk < 0) rk = 0;
+          }
+          const int s = kc % NS;
+          if (!mbar_wait(&bars->kv_empty[s], ((kc / NS) & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars->kv_full[s], C::kStage);
+          unsigned char* st = smem + C::kOffKV + s * C::kStage;
+          for (int x = 0; x < C::kHalves; ++x)
+            tma_load_2d(st + x * 8192, &tmk, x * 64, static_cast<int32_t>(rk), &bars->kv_full[s]);
+          for (int x = 0; x < C::kHalves; ++x)
+            tma_load_2d(st + C::kBlk + x * 8192, &tmv, x * 64, vrow0 + blk * kBlock,
+                        &bars->kv_full[s]);
         }
         if (!ok) break;
         ++un;
       }
       if (!ok) set_abort(bars, a.status);
       // copies in flight must land before the CTA exits (bounded)
-      for (uint32_t k = (kc > SK ? kc - SK : 0); k < kc; ++k)
-        mbar_wait(&bars->k_full[k % SK], (k / SK) & 1, 100000000ull);
+      for (uint32_t k = (kc > NS ? kc - NS : 0); k < kc; ++k)
+        mbar_wait(&bars->kv_full[k % NS], (k / NS) & 1, 100000000ull);
       if (un > 0) mbar_wait(&bars->q_full, (un - 1) & 1, 100000000ull);
     }
-  } else if (warp == kWarpLoadV) {
-    // ------------------------------------------------------------------ V loader
+  } else if (warp == kWarpMma0 || warp == kWarpMma0 + 1) {
+    // ------------------------------------------------- MMA issuer of tile t
+    const int t = warp - kWarpMma0;
     if (lane == 0) {
-      prefetch_tensormap(&tmv);
-      uint32_t un = 0, kc = 0;
-      bool ok = true;
-      while (ok) {
-        const int slot = un & 1;
-        if (!mbar_wait(&bars->info_full[slot], (un >> 1) & 1)) { ok = false; break; }
-        const UnitInfo U = bars->info[slot];
-        mbar_arrive(&bars->info_empty[slot]);
-        if (U.u < 0 || aborted(bars)) break;
-        const int npairs = (U.cnt + 1) / 2;
-        for (int pp = 0; pp < npairs; ++pp, ++kc) {
-          const int pi = kc % kPI;
-          // the pair's validated block ids come from the K loader
-          if (!mbar_wait(&bars->pi_full[pi], (kc / kPI) & 1)) { ok = false; break; }
-          const int4 P = bars->pinfo[pi];
-          mbar_arrive(&bars->pi_empty[pi]);
-          const int s = kc % SV;
-          if (!mbar_wait(&bars->v_empty[s], ((kc / SV) & 1) ^ 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars->v_full[s], P.z * C::kHalves * 8192);
-          unsigned char* vst = smem + C::kOffV + s * C::kTile;
-          for (int q = 0; q < P.z; ++q) {
-            const int blk = q == 0 ? P.x : P.y;
-            const int32_t rv = static_cast<int32_t>(
-                (static_cast<int64_t>(U.b) * a.Hkv + U.g) * a.Tpad + blk * kBlock);
-            for (int x = 0; x < C::kHalves; ++x)
-              tma_load_2d(vst + x * C::kSlab + q * 8192, &tmv, x * 64, rv, &bars->v_full[s]);
-          }
-        }
-        if (!ok) break;
-        ++un;
-      }
-      if (!ok) set_abort(bars, a.status);
-      for (uint32_t k = (kc > SV ? kc - SV : 0); k < kc; ++k)
-        mbar_wait(&bars->v_full[k % SV], (k / SV) & 1, 100000000ull);
-    }
-  } else if (warp == kWarpMma) {
-    // --------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idS128 = tc::idesc_f16(128, 128, 1, false);
-      const uint32_t idS64 = tc::idesc_f16(128, 64, 1, false);
+      const uint32_t idS = tc::idesc_f16(128, 64, 1, false);
       const uint32_t idPV = tc::idesc_f16(128, D, 0, true);
       const uint32_t sbase = smem_u32(smem);
+      const uint64_t dq = tc::smem_desc_sw128(sbase + t * C::kTile, 16, 1024);
+      const uint32_t o_tm = tmem + 128 * t, s_tm = tmem + 256 + 128 * t;
       uint32_t un = 0, kc = 0;
+      int s_left = 0;
       bool ok = true;
       while (ok) {
         const int slot = un & 1;
@@ -345,102 +304,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         const UnitInfo U = bars->info[slot];
         mbar_arrive(&bars->info_empty[slot]);
         if (U.u < 0 || aborted(bars)) break;
-        const int npairs = (U.cnt + 1) / 2;
+        if (t >= ntiles) { ++un; continue; }
+        const int n = U.cnt > 0 ? U.cnt : 1;
+        s_left = n;
         if (!mbar_wait(&bars->q_full, un & 1)) { ok = false; break; }
-        // Issue order per pair k (two tiles): S_0(k), P_1(k-1).V, S_1(k), P_0(k).V, so the
-        // softmax of one tile overlaps MMAs of the other. S_t(k) overwrites P_t(k-1): it
-        // waits for the P.V of tile t on pair k-1 (o_done). The P.V of tile 1 on a unit's
-        // last pair is issued when the unit ends.
-        int nk_prev = 0;
-        uint32_t sv_prev = 0;
-        for (int pp = 0; pp < npairs && ok; ++pp, ++kc) {
-          const int pi = kc % kPI;
-          if (!mbar_wait(&bars->pi_full[pi], (kc / kPI) & 1)) { ok = false; break; }
-          const int nk = bars->pinfo[pi].z * 64;
-          mbar_arrive(&bars->pi_empty[pi]);
-          const int sk = kc % SK, sv = kc % SV;
-          if (!mbar_wait(&bars->k_full[sk], (kc / SK) & 1)) { ok = false; break; }
-          const uint32_t kbase = sbase + C::kOffK + sk * C::kTile;
-          // ---- S_0(k)
-          if (kc > 0 && !mbar_wait(&bars->o_done[0], (kc - 1) & 1)) { ok = false; break; }
+        // S_t(j) into buffer j % 2 (last read by P_t(j-2).V)
+        auto issue_s = [&](uint32_t j) -> bool {
+          const int s = j % NS;
+          if (j >= 2 && !mbar_wait(&bars->pv_done[t][j & 1], ((j - 2) >> 1) & 1)) return false;
+          if (!mbar_wait(&bars->kv_full[s], (j / NS) & 1)) return false;
           tc::fence_after_sync();
+          const uint64_t dk = tc::smem_desc_sw128(sbase + C::kOffKV + s * C::kStage, 16, 1024);
 #pragma unroll
-          for (int ks = 0; ks < C::kKsteps; ++ks) {
-            const uint32_t off = (ks >> 2) * C::kSlab + (ks & 3) * 32;
-            tc::mma_ss(tmem, tc::smem_desc_sw128(sbase + off, 16, 1024),
-                       tc::smem_desc_sw128(kbase + off, 16, 1024), nk == 128 ? idS128 : idS64, ks > 0);
-          }
-          tc::commit(&bars->s_full[0]);
-          if (ntiles == 2) {
-            // ---- P_1(k-1).V  (same unit)
-            if (pp > 0) {
-              if (pp == 1 && un > 0 && !mbar_wait(&bars->o_free[1], (un - 1) & 1)) { ok = false; break; }
-              if (!mbar_wait(&bars->p_ready[1], (kc - 1) & 1)) { ok = false; break; }
-              tc::fence_after_sync();
-              for (int kk = 0; kk < nk_prev / 16; ++kk)
-                tc::mma_ts(tmem + 384, tmem + 128 + kk * 8,
-                           tc::smem_desc_sw128(sv_prev + kk * 2048, C::kSlab, 1024), idPV,
-                           pp > 1 || kk > 0);
-              tc::commit(&bars->o_done[1]);
-              tc::commit(&bars->v_empty[(kc - 1) % SV]);
-            }
-            // ---- S_1(k)
-            if (kc > 0 && !mbar_wait(&bars->o_done[1], (kc - 1) & 1)) { ok = false; break; }
-            tc::fence_after_sync();
-#pragma unroll
-            for (int ks = 0; ks < C::kKsteps; ++ks) {
-              const uint32_t off = (ks >> 2) * C::kSlab + (ks & 3) * 32;
-              tc::mma_ss(tmem + 128, tc::smem_desc_sw128(sbase + C::kTile + off, 16, 1024),
-                         tc::smem_desc_sw128(kbase + off, 16, 1024), nk == 128 ? idS128 : idS64,
-                         ks > 0);
-            }
-            tc::commit(&bars->s_full[1]);
-          }
-          tc::commit(&bars->k_empty[sk]);
-          if (pp == npairs - 1) tc::commit(&bars->q_empty);
-          // ---- P_0(k).V
-          if (!mbar_wait(&bars->v_full[sv], (kc / SV) & 1)) { ok = false; break; }
-          const uint32_t vbase = sbase + C::kOffV + sv * C::kTile;
-          if (pp == 0 && un > 0 && !mbar_wait(&bars->o_free[0], (un - 1) & 1)) { ok = false; break; }
-          if (!mbar_wait(&bars->p_ready[0], kc & 1)) { ok = false; break; }
+          for (int ks = 0; ks < C::kKsteps; ++ks)
+            tc::mma_ss(s_tm + 64 * (j & 1), dq + (((ks >> 2) * C::kSlab + (ks & 3) * 32) >> 4),
+                       dk + (((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), idS, ks > 0);
+          tc::commit(&bars->s_full[t][j & 1]);
+          if (--s_left == 0) tc::commit(&bars->q_empty);
+          return true;
+        };
+        // O_t += P_t(j) V_j; the first step of a unit overwrites O once the epilogue of
+        // the previous unit has read it
+        auto issue_pv = [&](uint32_t j, bool first) -> bool {
+          const int s = j % NS;
+          if (first && un > 0 && !mbar_wait(&bars->o_free[t], (un - 1) & 1)) return false;
+          if (!mbar_wait(&bars->p_ready[t][j & 1], (j >> 1) & 1)) return false;
           tc::fence_after_sync();
-          for (int kk = 0; kk < nk / 16; ++kk)
-            tc::mma_ts(tmem + 256, tmem + kk * 8, tc::smem_desc_sw128(vbase + kk * 2048, C::kSlab, 1024),
-                       idPV, pp > 0 || kk > 0);
-          tc::commit(&bars->o_done[0]);
-          if (ntiles == 1) tc::commit(&bars->v_empty[sv]);
-          nk_prev = nk;
-          sv_prev = vbase;
+          const uint64_t dv =
+              tc::smem_desc_sw128(sbase + C::kOffKV + s * C::kStage + C::kBlk, 8192, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc::mma_ts(o_tm, s_tm + 64 * (j & 1) + kk * 8, dv + ((kk * 2048) >> 4), idPV,
+                       !first || kk > 0);
+          tc::commit(&bars->pv_done[t][j & 1]);
+          tc::commit(&bars->kv_empty[s]);
+          return true;
+        };
+        ok = issue_s(kc) && (n < 2 || issue_s(kc + 1));
+        for (int jj = 0; jj < n && ok; ++jj) {
+          ok = issue_pv(kc + jj, jj == 0);
+          if (ok && jj + 2 < n) ok = issue_s(kc + jj + 2);
         }
         if (!ok) break;
-        if (ntiles == 2) {
-          // ---- P_1(last).V
-          if (npairs == 1 && un > 0 && !mbar_wait(&bars->o_free[1], (un - 1) & 1)) { ok = false; break; }
-          if (!mbar_wait(&bars->p_ready[1], (kc - 1) & 1)) { ok = false; break; }
-          tc::fence_after_sync();
-          for (int kk = 0; kk < nk_prev / 16; ++kk)
-            tc::mma_ts(tmem + 384, tmem + 128 + kk * 8,
-                       tc::smem_desc_sw128(sv_prev + kk * 2048, C::kSlab, 1024), idPV,
-                       npairs > 1 || kk > 0);
-          tc::commit(&bars->o_done[1]);
-          tc::commit(&bars->v_empty[(kc - 1) % SV]);
-        }
-        if (!ok) break;
+        kc += n;
         ++un;
       }
       if (!ok) set_abort(bars, a.status);
-      // every MMA issued so far must finish before tensor memory is freed (bounded)
-      tc::commit(&bars->mma_done);
-      mbar_wait(&bars->mma_done, 0, 200000000ull);
+      // every MMA this thread issued must finish before tensor memory is freed (bounded)
+      tc::commit(&bars->mma_done[t]);
+      mbar_wait(&bars->mma_done[t], 0, 200000000ull);
     }
   } else if (warp >= kWarpSm0) {
     // ----------------------------------------------------------- softmax warps
-    const int t = (warp - kWarpSm0) >> 2;
+    // 8 warps per tile: warp w owns the 16 rows [32*(w%4) + 16*h, +16) of its tile
+    // (w % 4 is the tensor-memory lane quarter it may access, h its half of it).
+    // Thread (t0 = lane % 4, t1 = lane / 4) holds rows t1 and t1 + 8 of those 16 and,
+    // of each 8-column group k, columns 8k + 2*t0 and 8k + 2*t0 + 1 (the .16x256b
+    // layout); its packed fp16 P pair of those columns lands in P column 4k + t0
+    // (.16x128b), which is where the P.V MMA reads keys 8k + 2*t0, +1 of the row.
+    const int t = (warp - kWarpSm0) >> 3;
+    const int hseg = ((warp - kWarpSm0) >> 2) & 1;
     const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;
-    const uint32_t lane_addr = static_cast<uint32_t>(q4 * 32) << 16;
-    const uint32_t s_col = tmem + lane_addr + 128 * t;
-    const uint32_t o_col = tmem + lane_addr + 256 + 128 * t;
+    const int t0 = lane & 3, t1 = lane >> 2;
+    const int rbase = q4 * 32 + hseg * 16;
+    const int ra = rbase + t1, rb = ra + 8;
+    const uint32_t lane_addr = static_cast<uint32_t>(rbase) << 16;
+    const uint32_t s_col0 = tmem + lane_addr + 256 + 128 * t;
+    const uint32_t o_col = tmem + lane_addr + 128 * t;
     const float sc = a.scale_log2;
     const float2 sc2 = make_float2(sc, sc);
     uint32_t un = 0, kc = 0;
@@ -456,139 +386,182 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++un;
       if (U.u < 0) break;
       if (t >= ntiles) continue;
-      const int npairs = (U.cnt + 1) / 2;
-      const int tq = U.i * kBlock + (r & 63);
-      float m = -INFINITY;
-      float2 l2 = make_float2(0.f, 0.f);
+      const int n = U.cnt > 0 ? U.cnt : 1;
+      const int32_t* klist =
+          a.kept + (static_cast<int64_t>(U.b * a.Hkv + U.g) * a.nqb + U.i) * a.max_kept;
+      const int tqa = U.i * kBlock + (ra & 63), tqb = U.i * kBlock + (rb & 63);
+      float ma = -INFINITY, mb = -INFINITY;
+      float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
+      // block id and mask mode of the current step (the next one is fetched a step ahead)
+      int blk = U.i, mode = 2;
+      if (U.cnt > 0) {
+        blk = klist[0];
+        mode = mode_of(a, U, blk);
+      }
       bool ok = true;
-      for (int pp = 0; pp < npairs; ++pp, ++kc) {
-        const int pi = kc % kPI;
-        if (!warp_wait(&bars->pi_full[pi], (kc / kPI) & 1)) { ok = false; break; }
-        const int4 P = bars->pinfo[pi];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->pi_empty[pi]);
-        if (!warp_wait(&bars->s_full[t], kc & 1)) { ok = false; break; }
+      for (int jj = 0; jj < n; ++jj, ++kc) {
+        const int blk_nx = jj + 1 < U.cnt ? klist[jj + 1] : U.i;
+        const int buf = kc & 1;
+        if (!warp_wait(&bars->s_full[t][buf], (kc >> 1) & 1)) { ok = false; break; }
         tc::fence_after_sync();
-        const int nb = P.z;
-        const int mode0 = P.w & 0xff, mode1 = (P.w >> 8) & 0xff;
-        // S row of this thread: chunks of 32 columns (block q = chunks 2q, 2q+1)
-        uint32_t r[4][32];
-        tc::ld32(s_col, r[0]);
-        tc::ld32(s_col + 32, r[1]);
-        if (nb == 2) {
-          tc::ld32(s_col + 64, r[2]);
-          tc::ld32(s_col + 96, r[3]);
-        }
+        const uint32_t s_col = s_col0 + 64 * buf;
+        uint32_t sr[32];
+        tc::ld16x256_x8(s_col, sr);
         tc::wait_ld();
-        // masks: the causal diagonal block, and blocks that failed validation
-        if (mode0 != 0) mask_block(r[0], r[1], mode0 == 2 ? -1 : tq - P.x * kBlock);
-        if (nb == 2 && mode1 != 0) mask_block(r[2], r[3], mode1 == 2 ? -1 : tq - P.y * kBlock);
-        float mx = -INFINITY;
+        // masks: the causal diagonal block and blocks that failed validation
+        if (mode != 0) {
+          const int dblk = mode == 2 ? 0 : blk;
+          const int lima = mode == 2 ? -1 : tqa - dblk * kBlock;
+          const int limb = mode == 2 ? -1 : tqb - dblk * kBlock;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < 2 * nb) {
-#pragma unroll
-            for (int x = 0; x < 32; x += 2)
-              mx = max3(mx, __uint_as_float(r[c][x]), __uint_as_float(r[c][x + 1]));
+          for (int k = 0; k < 8; ++k) {
+            const int c = k * 8 + 2 * t0;   // column within the block
+            if (c > lima) sr[4 * k] = 0xff800000u;
+            if (c + 1 > lima) sr[4 * k + 1] = 0xff800000u;
+            if (c > limb) sr[4 * k + 2] = 0xff800000u;
+            if (c + 1 > limb) sr[4 * k + 3] = 0xff800000u;
           }
         }
-        mx *= sc;
-        if (mx > m + 8.0f) {
-          // move the running max: rescale l and the O row accumulated so far
-          const float f = ex2(m - mx);
-          l2.x *= f;
-          l2.y *= f;
-          if (pp > 0) {
+        // row maxima (each row spans the 4 threads with the same t1): two chains per row
+        float xa = -INFINITY, xa2 = -INFINITY, xb = -INFINITY, xb2 = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+          xa = max3(xa, __uint_as_float(sr[4 * k]), __uint_as_float(sr[4 * k + 1]));
+          xa2 = max3(xa2, __uint_as_float(sr[4 * k + 4]), __uint_as_float(sr[4 * k + 5]));
+          xb = max3(xb, __uint_as_float(sr[4 * k + 2]), __uint_as_float(sr[4 * k + 3]));
+          xb2 = max3(xb2, __uint_as_float(sr[4 * k + 6]), __uint_as_float(sr[4 * k + 7]));
+        }
+        xa = fmaxf(xa, xa2);
+        xb = fmaxf(xb, xb2);
+        xa = fmaxf(xa, __shfl_xor_sync(0xffffffffu, xa, 1));
+        xb = fmaxf(xb, __shfl_xor_sync(0xffffffffu, xb, 1));
+        xa = fmaxf(xa, __shfl_xor_sync(0xffffffffu, xa, 2));
+        xb = fmaxf(xb, __shfl_xor_sync(0xffffffffu, xb, 2));
+        xa *= sc;
+        xb *= sc;
+        const bool upa = xa > ma + 8.0f, upb = xb > mb + 8.0f;
+        // move the running max of the rows that need it (O is rescaled below, after P)
+        const bool any_up = __any_sync(0xffffffffu, upa || upb);
+        const float fa = upa ? ex2(ma - xa) : 1.0f;
+        const float fb = upb ? ex2(mb - xb) : 1.0f;
+        if (upa) {
+          la.x *= fa;
+          la.y *= fa;
+          ma = xa;
+        }
+        if (upb) {
+          lb.x *= fb;
+          lb.y *= fb;
+          mb = xb;
+        }
+        const float na = ma == -INFINITY ? 0.f : -ma, nbb = mb == -INFINITY ? 0.f : -mb;
+        const float2 na2 = make_float2(na, na), nb2 = make_float2(nbb, nbb);
+        // P = 2^(s * scale - m) in fp16, packed in place (word 2k: row a, 2k+1: row b)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float2 va = __ffma2_rn(make_float2(__uint_as_float(sr[4 * k]), __uint_as_float(sr[4 * k + 1])), sc2, na2);
+          const float2 vb = __ffma2_rn(make_float2(__uint_as_float(sr[4 * k + 2]), __uint_as_float(sr[4 * k + 3])), sc2, nb2);
+          float2 pa, pb;
+          if (k >= 8 - kPolyGroups) {
+            pa = exp2_poly(va);
+            pb = exp2_poly(vb);
+          } else {
+            pa = make_float2(ex2(va.x), ex2(va.y));
+            pb = make_float2(ex2(vb.x), ex2(vb.y));
+          }
+          la = __fadd2_rn(la, pa);
+          lb = __fadd2_rn(lb, pb);
+          sr[2 * k] = pack_f16(pa.x, pa.y);
+          sr[2 * k + 1] = pack_f16(pb.x, pb.y);
+        }
+        tc::st16x128_x8(s_col, *reinterpret_cast<const uint32_t(*)[16]>(&sr[0]));
+        if (any_up && jj > 0) {
+          // rescale the O rows accumulated so far (warp-wide: tcgen05.ld/st are
+          // collective), once the P.V of the previous step has completed
+          const uint32_t jp = kc - 1;
+          if (!warp_wait(&bars->pv_done[t][jp & 1], (jp >> 1) & 1)) { ok = false; break; }
+          tc::fence_after_sync();
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t ov[32];
-              tc::ld32(o_col + c * 32, ov);
-              tc::wait_ld();
+          for (int half = 0; half < D / 64; ++half) {
+            uint32_t ov[32];
+            tc::ld16x256_x8(o_col + 64 * half, ov);
+            tc::wait_ld();
 #pragma unroll
-              for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * f);
-              tc::st32(o_col + c * 32, ov);
+            for (int k = 0; k < 8; ++k) {
+              ov[4 * k] = __float_as_uint(__uint_as_float(ov[4 * k]) * fa);
+              ov[4 * k + 1] = __float_as_uint(__uint_as_float(ov[4 * k + 1]) * fa);
+              ov[4 * k + 2] = __float_as_uint(__uint_as_float(ov[4 * k + 2]) * fb);
+              ov[4 * k + 3] = __float_as_uint(__uint_as_float(ov[4 * k + 3]) * fb);
             }
-            tc::wait_st();
-          }
-          m = mx;
-        }
-        const float nbase = m == -INFINITY ? 0.f : -m;
-        const float2 nb2 = make_float2(nbase, nbase);
-        // P = 2^(s * scale - m) in fp16, packed in place over the consumed S values
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c < 2 * nb) {
-#pragma unroll
-            for (int x = 0; x < 16; ++x) {
-              const float2 s2 = make_float2(__uint_as_float(r[c][2 * x]), __uint_as_float(r[c][2 * x + 1]));
-              const float2 xv = __ffma2_rn(s2, sc2, nb2);
-              float2 p;
-              if (x >= 16 - kPolyPairs) {
-                p = exp2_poly(xv);
-              } else {
-                p.x = ex2(xv.x);
-                p.y = ex2(xv.y);
-              }
-              l2 = __fadd2_rn(l2, p);
-              r[c][x] = pack_f16(p.x, p.y);
-            }
-            tc::st16(s_col + 16 * c, *reinterpret_cast<const uint32_t(*)[16]>(&r[c][0]));
+            tc::st16x256_x8(o_col + 64 * half, ov);
           }
         }
         tc::wait_st();
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_ready[t]);
+        if (lane == 0) mbar_arrive(&bars->p_ready[t][buf]);
+        blk = blk_nx;
+        mode = jj + 1 < U.cnt ? mode_of(a, U, blk) : 2;
       }
       if (!ok || aborted(bars)) {
         if (lane == 0) set_abort(bars, a.status);
         break;
       }
-      // ---- epilogue: O / l
-      if (!warp_wait(&bars->o_done[t], (kc - 1) & 1)) {
+      // ---- epilogue: O / l, once the unit's last P.V has completed
+      const uint32_t jl = kc - 1;
+      if (!warp_wait(&bars->pv_done[t][jl & 1], (jl >> 1) & 1)) {
         if (lane == 0) set_abort(bars, a.status);
         break;
       }
       tc::fence_after_sync();
-      const float l = l2.x + l2.y;
-      const int hl = row_head(a, U.hq, t, r);
-      const bool write = tq < a.T && (4 * U.hq + 2 * t + (r >> 6)) < a.G;
-      const int64_t hrow = (static_cast<int64_t>(U.b) * a.Hq + U.g * a.G + hl) * a.T + tq;
-      const float inv = l > 0.f ? 1.0f / l : 0.f;
+      float La = la.x + la.y, Lb = lb.x + lb.y;
+      La += __shfl_xor_sync(0xffffffffu, La, 1);
+      La += __shfl_xor_sync(0xffffffffu, La, 2);
+      Lb += __shfl_xor_sync(0xffffffffu, Lb, 1);
+      Lb += __shfl_xor_sync(0xffffffffu, Lb, 2);
+      const float inva = La > 0.f ? 1.0f / La : 0.f, invb = Lb > 0.f ? 1.0f / Lb : 0.f;
+      const bool wa = tqa < a.T && (4 * U.hq + 2 * t + (ra >> 6)) < a.G;
+      const bool wb = tqb < a.T && (4 * U.hq + 2 * t + (rb >> 6)) < a.G;
+      const int64_t hra =
+          (static_cast<int64_t>(U.b) * a.Hq + U.g * a.G + row_head(a, U.hq, t, ra)) * a.T + tqa;
+      const int64_t hrb =
+          (static_cast<int64_t>(U.b) * a.Hq + U.g * a.G + row_head(a, U.hq, t, rb)) * a.T + tqb;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int half = 0; half < D / 64; ++half) {
         uint32_t ov[32];
-        tc::ld32(o_col + c * 32, ov);
+        tc::ld16x256_x8(o_col + 64 * half, ov);
         tc::wait_ld();
-        if (write) {
-          uint32_t pk[16];
 #pragma unroll
-          for (int x = 0; x < 16; ++x)
-            pk[x] = pack_bf16(__uint_as_float(ov[2 * x]) * inv, __uint_as_float(ov[2 * x + 1]) * inv);
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + hrow * D + c * 32);
+        for (int rr = 0; rr < 2; ++rr) {
+          if (rr ? wb : wa) {
+            const int64_t hrow = rr ? hrb : hra;
+            const float inv = rr ? invb : inva;
+            __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o) + hrow * D + 64 * half;
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
-          if (a.o_f32) {
-            float4* df = reinterpret_cast<float4*>(a.o_f32 + hrow * D + c * 32);
-#pragma unroll
-            for (int x = 0; x < 8; ++x)
-              df[x] = make_float4(__uint_as_float(ov[4 * x]) * inv, __uint_as_float(ov[4 * x + 1]) * inv,
-                                  __uint_as_float(ov[4 * x + 2]) * inv,
-                                  __uint_as_float(ov[4 * x + 3]) * inv);
+            for (int k = 0; k < 8; ++k) {
+              const float v0 = __uint_as_float(ov[4 * k + 2 * rr]) * inv;
+              const float v1 = __uint_as_float(ov[4 * k + 2 * rr + 1]) * inv;
+              *reinterpret_cast<__nv_bfloat162*>(ob + 8 * k + 2 * t0) = __floats2bfloat162_rn(v0, v1);
+              if (a.o_f32)
+                *reinterpret_cast<float2*>(a.o_f32 + hrow * D + 64 * half + 8 * k + 2 * t0) =
+                    make_float2(v0, v1);
+            }
           }
         }
       }
-      if (write) a.lse[hrow] = l > 0.f ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      if (t0 == 0) {
+        if (wa) a.lse[hra] = La > 0.f ? (ma + log2f(La)) * 0.69314718055994530942f : -INFINITY;
+        if (wb) a.lse[hrb] = Lb > 0.f ? (mb + log2f(Lb)) * 0.69314718055994530942f : -INFINITY;
+      }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->o_free[t]);
+      if (lane == 0) mbar_arrive(&bars->o_free[t]);   // O of this tile may be overwritten now
     }
   }
 
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == kWarpMma) {
+  if (warp == kWarpMma0) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
