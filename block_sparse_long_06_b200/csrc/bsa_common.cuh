@@ -86,7 +86,7 @@ BSA_DEVFN bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hi
 // where spinning warps would take issue slots from the warps doing the work.
 BSA_DEVFN bool mbar_wait_sleep(uint64_t* bar, uint32_t parity,
                                uint64_t limit_ns = 2000000000ull) {
-  if (mbar_try_wait_suspend(bar, parity, 100000u)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait_suspend(bar, parity, 100000u)) return true;

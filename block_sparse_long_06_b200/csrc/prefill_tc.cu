@@ -14,16 +14,15 @@
 //  * a step is one kept key block (64 keys) for both tiles. Warp 0 (one lane)
 //    loads Q once per unit and, per step, the K block (bf16) and the V block (fp16)
 //    into one stage of a K/V ring (TMA, 128-byte swizzle);
-//  * one MMA-issuing thread per tile (warps 1 and 2): a single thread can issue a
-//    tcgen05.mma only every ~50 cycles and a commit costs about as much, so one
-//    issuer for both tiles would leave the tensor core idle. Tile t's issuer runs
-//    S_t(j) = Q_t K_j^T (bf16, M = 128, N = 64, K = d) into one of the tile's two S
-//    buffers in tensor memory and O_t += P_t(j) V_j (fp16, P read from tensor
-//    memory over the S columns, N = d), in the order P_t(j).V, S_t(j+2): the score
-//    MMAs run two steps ahead, so the softmax of a tile goes from one step to the
-//    next without waiting for the tensor core. An S buffer is reused once the
-//    P.V that read it has completed; a K/V stage is released by the P.V of every
-//    tile;
+//  * three MMA-issuing threads (warps 1-2: scores of tile 0/1, warp 3: P.V of both
+//    tiles): a single thread can issue a tcgen05.mma only every ~50 cycles and a
+//    commit costs about as much, so one issuer would leave the tensor core idle. S_t(j) = Q_t K_j^T (bf16, M = 128,
+//    N = 64, K = d) goes to one of the tile's two S buffers in tensor memory;
+//    O_t += P_t(j) V_j (fp16, P read from tensor memory over the S columns, N = d).
+//    The score MMAs run up to two steps ahead of the P.V, so the softmax of a tile
+//    goes from one step to the next without waiting for the tensor core. An S
+//    buffer is reused once the P.V that read it has completed; a K/V stage is
+//    released by the P.V of every tile;
 //  * warps 4-11 and 12-19 are the softmax warps of tile 0 and tile 1, 16 rows each
 //    (tensor-memory lane quarter = warp % 4). They read the step's block id from
 //    the kept list and validate it themselves, so the only per-step wait is for S.
@@ -48,7 +47,11 @@ namespace bsa {
 namespace {
 
 constexpr int kThreads = 640;
-constexpr int kWarpLoad = 0, kWarpMma0 = 1, kWarpSm0 = 4;
+// warp roles: loader, score-MMA issuers of tiles 0/1, the P.V issuer of both tiles, and
+// the 16 softmax warps 4-19 (a softmax warp's tensor-memory lane quarter is warp % 4).
+// 20 warps = 5 per SM sub-partition, which leaves 96 registers a thread.
+constexpr int kWarpLoad = 0, kWarpS0 = 1, kWarpPV = 3, kWarpSm0 = 4;
+constexpr int kIssuers = 3;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxStages = 8;
 constexpr int kPolyGroups = 3;  // of every 8 column groups of a row: exponentials by polynomial
@@ -76,7 +79,7 @@ struct Bars {
   uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
   uint64_t s_full[2][2], p_ready[2][2], pv_done[2][2];   // [tile][S buffer]
   uint64_t o_free[2];
-  uint64_t mma_done[2];
+  uint64_t mma_done[kIssuers];
   UnitInfo info[2];
   uint32_t tmem_base;
   int abort_flag;
@@ -193,25 +196,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->info_full[x], 1);
-      mbar_init(&bars->info_empty[x], 2 + 16);    // both issuers, every softmax warp
+      mbar_init(&bars->info_empty[x], kIssuers + 16);   // every issuer and softmax warp
       for (int y = 0; y < 2; ++y) {
         mbar_init(&bars->s_full[x][y], 1);
         mbar_init(&bars->p_ready[x][y], 8);       // the 8 softmax warps of a tile
         mbar_init(&bars->pv_done[x][y], 1);
       }
       mbar_init(&bars->o_free[x], 8);
-      mbar_init(&bars->mma_done[x], 1);
     }
+    for (int x = 0; x < kIssuers; ++x) mbar_init(&bars->mma_done[x], 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], ntiles);      // the P.V of every tile
+      mbar_init(&bars->kv_empty[s], 1);           // after the P.V of every tile
     }
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, ntiles);            // the last score MMAs of every tile
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kWarpMma0) {
+  if (warp == kWarpS0) {
     tc::tmem_alloc(&bars->tmem_base, kTmemCols);
     tc::tmem_relinquish();
   }
@@ -286,17 +289,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&bars->kv_full[k % NS], (k / NS) & 1, 100000000ull);
       if (un > 0) mbar_wait(&bars->q_full, (un - 1) & 1, 100000000ull);
     }
-  } else if (warp == kWarpMma0 || warp == kWarpMma0 + 1) {
-    // ------------------------------------------------- MMA issuer of tile t
-    const int t = warp - kWarpMma0;
+  } else if (warp == kWarpS0 || warp == kWarpS0 + 1) {
+    // ------------------------------------------ score-MMA issuer of tile t
+    // S_t(j) = Q_t K_j^T into S buffer j % 2, once P_t(j-2).V (the last reader of
+    // that buffer) has completed; at most two steps ahead of the P.V issuer.
+    const int t = warp - kWarpS0;
     if (lane == 0) {
       const uint32_t idS = tc::idesc_f16(128, 64, 1, false);
-      const uint32_t idPV = tc::idesc_f16(128, D, 0, true);
       const uint32_t sbase = smem_u32(smem);
       const uint64_t dq = tc::smem_desc_sw128(sbase + t * C::kTile, 16, 1024);
-      const uint32_t o_tm = tmem + 128 * t, s_tm = tmem + 256 + 128 * t;
+      const uint32_t s_tm = tmem + 256 + 128 * t;
       uint32_t un = 0, kc = 0;
-      int s_left = 0;
       bool ok = true;
       while (ok) {
         const int slot = un & 1;
@@ -306,13 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (U.u < 0 || aborted(bars)) break;
         if (t >= ntiles) { ++un; continue; }
         const int n = U.cnt > 0 ? U.cnt : 1;
-        s_left = n;
         if (!mbar_wait(&bars->q_full, un & 1)) { ok = false; break; }
-        // S_t(j) into buffer j % 2 (last read by P_t(j-2).V)
-        auto issue_s = [&](uint32_t j) -> bool {
+        for (int jj = 0; jj < n; ++jj) {
+          const uint32_t j = kc + jj;
           const int s = j % NS;
-          if (j >= 2 && !mbar_wait(&bars->pv_done[t][j & 1], ((j - 2) >> 1) & 1)) return false;
-          if (!mbar_wait(&bars->kv_full[s], (j / NS) & 1)) return false;
+          if (j >= 2 && !mbar_wait(&bars->pv_done[t][j & 1], ((j - 2) >> 1) & 1)) { ok = false; break; }
+          if (!mbar_wait(&bars->kv_full[s], (j / NS) & 1)) { ok = false; break; }
           tc::fence_after_sync();
           const uint64_t dk = tc::smem_desc_sw128(sbase + C::kOffKV + s * C::kStage, 16, 1024);
 #pragma unroll
@@ -320,32 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mma_ss(s_tm + 64 * (j & 1), dq + (((ks >> 2) * C::kSlab + (ks & 3) * 32) >> 4),
                        dk + (((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), idS, ks > 0);
           tc::commit(&bars->s_full[t][j & 1]);
-          if (--s_left == 0) tc::commit(&bars->q_empty);
-          return true;
-        };
-        // O_t += P_t(j) V_j; the first step of a unit overwrites O once the epilogue of
-        // the previous unit has read it
-        auto issue_pv = [&](uint32_t j, bool first) -> bool {
-          const int s = j % NS;
-          if (first && un > 0 && !mbar_wait(&bars->o_free[t], (un - 1) & 1)) return false;
-          if (!mbar_wait(&bars->p_ready[t][j & 1], (j >> 1) & 1)) return false;
-          tc::fence_after_sync();
-          const uint64_t dv =
-              tc::smem_desc_sw128(sbase + C::kOffKV + s * C::kStage + C::kBlk, 8192, 1024);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc::mma_ts(o_tm, s_tm + 64 * (j & 1) + kk * 8, dv + ((kk * 2048) >> 4), idPV,
-                       !first || kk > 0);
-          tc::commit(&bars->pv_done[t][j & 1]);
-          tc::commit(&bars->kv_empty[s]);
-          return true;
-        };
-        ok = issue_s(kc) && (n < 2 || issue_s(kc + 1));
-        for (int jj = 0; jj < n && ok; ++jj) {
-          ok = issue_pv(kc + jj, jj == 0);
-          if (ok && jj + 2 < n) ok = issue_s(kc + jj + 2);
         }
         if (!ok) break;
+        tc::commit(&bars->q_empty);   // Q of this tile is free once these MMAs complete
         kc += n;
         ++un;
       }
@@ -354,7 +333,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::commit(&bars->mma_done[t]);
       mbar_wait(&bars->mma_done[t], 0, 200000000ull);
     }
-  } else if (warp >= kWarpSm0) {
+  } else if (warp == kWarpPV) {
+    // ------------------------------------------- P.V issuer of both tiles
+    // O_t += P_t(j) V_j once the softmax has written P_t(j); the first step of a unit
+    // overwrites O once the epilogue of the previous unit has read it. The commit on
+    // kv_empty releases the K/V stage (its S MMAs completed before P was written).
+    if (lane == 0) {
+      const uint32_t idPV = tc::idesc_f16(128, D, 0, true);
+      const uint32_t sbase = smem_u32(smem);
+      uint32_t un = 0, kc = 0;
+      bool ok = true;
+      while (ok) {
+        const int slot = un & 1;
+        if (!mbar_wait(&bars->info_full[slot], (un >> 1) & 1)) { ok = false; break; }
+        const UnitInfo U = bars->info[slot];
+        mbar_arrive(&bars->info_empty[slot]);
+        if (U.u < 0 || aborted(bars)) break;
+        const int n = U.cnt > 0 ? U.cnt : 1;
+        for (int jj = 0; jj < n && ok; ++jj) {
+          const uint32_t j = kc + jj;
+          const int s = j % NS;
+          const uint64_t dv =
+              tc::smem_desc_sw128(sbase + C::kOffKV + s * C::kStage + C::kBlk, 8192, 1024);
+          for (int t = 0; t < ntiles; ++t) {
+            if (jj == 0 && un > 0 && !mbar_wait(&bars->o_free[t], (un - 1) & 1)) { ok = false; break; }
+            if (!mbar_wait(&bars->p_ready[t][j & 1], (j >> 1) & 1)) { ok = false; break; }
+            tc::fence_after_sync();
+            const uint32_t o_tm = tmem + 128 * t, p_tm = tmem + 256 + 128 * t + 64 * (j & 1);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tc::mma_ts(o_tm, p_tm + kk * 8, dv + ((kk * 2048) >> 4), idPV, jj > 0 || kk > 0);
+            tc::commit(&bars->pv_done[t][j & 1]);
+          }
+          if (ok) tc::commit(&bars->kv_empty[s]);
+        }
+        if (!ok) break;
+        kc += n;
+        ++un;
+      }
+      if (!ok) set_abort(bars, a.status);
+      tc::commit(&bars->mma_done[2]);
+      mbar_wait(&bars->mma_done[2], 0, 200000000ull);
+    }
+  } else if (warp >= kWarpSm0 && warp < kWarpSm0 + 16) {
     // ----------------------------------------------------------- softmax warps
     // 8 warps per tile: warp w owns the 16 rows [32*(w%4) + 16*h, +16) of its tile
     // (w % 4 is the tensor-memory lane quarter it may access, h its half of it).
@@ -561,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == kWarpMma0) {
+  if (warp == kWarpS0) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
