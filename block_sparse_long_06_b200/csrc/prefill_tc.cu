@@ -19,9 +19,10 @@
 //    commit costs about as much, so one issuer would leave the tensor core idle. S_t(j) = Q_t K_j^T (bf16, M = 128,
 //    N = 64, K = d) goes to one of the tile's two S buffers in tensor memory;
 //    O_t += P_t(j) V_j (fp16, P read from tensor memory over the S columns, N = d).
-//    The score MMAs run up to two steps ahead of the P.V, so the softmax of a tile
-//    goes from one step to the next without waiting for the tensor core. An S
-//    buffer is reused once the P.V that read it has completed; a K/V stage is
+//    P has tensor-memory buffers of its own (two per tile), so the S buffer of a
+//    tile is free as soon as its softmax warps have loaded S into registers: the
+//    score MMAs of step j+1 run while the softmax of step j computes, and the P.V
+//    is off that loop (a P buffer is reused two steps later). A K/V stage is
 //    released by the P.V of every tile;
 //  * warps 4-11 and 12-19 are the softmax warps of tile 0 and tile 1, 16 rows each
 //    (tensor-memory lane quarter = warp % 4). They read the step's block id from
@@ -29,15 +30,15 @@
 //    A thread holds 2 rows x 16 columns of S, masks the causal diagonal block (and
 //    blocks that failed validation), takes the row max (three-input max, then 2
 //    shuffles), computes P with packed two-wide fp32 arithmetic and writes it as
-//    fp16 over the S columns. 3/8 of the exponentials run as a cubic polynomial on
+//    fp16 to the P buffer. 3/8 of the exponentials run as a cubic polynomial on
 //    the FMA pipes (exp2_poly below) instead of the MUFU unit. The running max only
 //    moves (and O is rescaled in tensor memory, after the previous P.V has
 //    completed) when it grows by more than 8 (log2), so P <= 256 fits fp16 and the
 //    rescale is rare; the final normalisation uses the same max, so it is exact;
 //  * epilogue: O / l from tensor memory straight to global memory (bf16, and fp32
 //    when requested), LSE in natural log.
-// Tensor memory: 512 columns: O of tile t at 128 t; S/P buffer b of tile t at
-// 256 + 128 t + 64 b. Every wait is bounded; on a timeout the kernel sets
+// Tensor memory: 512 columns: O of tile t at 128 t, S of tile t at 256 + 64 t, P
+// buffer b of tile t at 384 + 64 t + 32 b. Every wait is bounded; on a timeout the kernel sets
 // BSA_DEV_TIMEOUT, drains, frees its tensor memory and returns.
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
@@ -77,7 +78,8 @@ struct Bars {
   uint64_t info_full[2], info_empty[2];
   uint64_t q_full, q_empty;
   uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
-  uint64_t s_full[2][2], p_ready[2][2], pv_done[2][2];   // [tile][S buffer]
+  uint64_t s_full[2], s_free[2];                        // [tile]
+  uint64_t p_ready[2][2], pv_done[2][2];                 // [tile][P buffer]
   uint64_t o_free[2];
   uint64_t mma_done[kIssuers];
   UnitInfo info[2];
@@ -112,8 +114,10 @@ BSA_DEVFN UnitInfo unit_of(const PrefillArgs& a, int u) {
   return U;
 }
 
-// Row of the first token of block `blk` (rows of width d) or -1 when invalid.
-BSA_DEVFN int64_t krow_of(const CacheView& c, const PrefillArgs& a, int b, int g, int blk, int i) {
+// Element offset of the first token of block `blk` in cache `c`, or -1 when the block
+// is not a valid kept block of query block i (out of range, bad page, past the extent).
+BSA_DEVFN int64_t block_off(const CacheView& c, const PrefillArgs& a, int b, int g, int blk,
+                            int i) {
   if (blk < 0 || blk > i) return -1;
   int64_t phys = blk;
   if (c.page_table != nullptr) {
@@ -124,7 +128,13 @@ BSA_DEVFN int64_t krow_of(const CacheView& c, const PrefillArgs& a, int b, int g
   const int64_t off = static_cast<int64_t>(b) * c.seq_stride + phys * c.block_stride +
                       static_cast<int64_t>(g) * c.head_stride;
   if (off < 0 || off + static_cast<int64_t>(rows) * a.d > c.extent) return -1;
-  return off / a.d;
+  return off;
+}
+
+// Row of the first token of block `blk` (rows of width d) or -1 when invalid.
+BSA_DEVFN int64_t krow_of(const CacheView& c, const PrefillArgs& a, int b, int g, int blk, int i) {
+  const int64_t off = block_off(c, a, b, g, blk, i);
+  return off < 0 ? -1 : off / a.d;
 }
 
 // Head (within the group) of row r of tile t of head quad hq (clamped for G < 4).
@@ -137,7 +147,7 @@ BSA_DEVFN int row_head(const PrefillArgs& a, int hq, int t, int r) {
 // (Polling from every lane only adds shared-memory traffic.)
 BSA_DEVFN bool warp_wait(uint64_t* bar, uint32_t parity) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait_sleep(bar, parity);
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
@@ -174,7 +184,7 @@ BSA_DEVFN float2 exp2_poly(float2 x) {
 // Mask mode of a kept block: 0 visible, 1 the causal diagonal, 2 failed validation
 // (the loader then loads the diagonal block in its place).
 BSA_DEVFN int mode_of(const PrefillArgs& a, const UnitInfo& U, int blk) {
-  if (krow_of(a.k, a, U.b, U.g, blk, U.i) < 0) return 2;
+  if (block_off(a.k, a, U.b, U.g, blk, U.i) < 0) return 2;
   return blk == U.i ? 1 : 0;
 }
 
@@ -197,9 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->info_full[x], 1);
       mbar_init(&bars->info_empty[x], kIssuers + 16);   // every issuer and softmax warp
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->s_free[x], 8);             // the 8 softmax warps of a tile
       for (int y = 0; y < 2; ++y) {
-        mbar_init(&bars->s_full[x][y], 1);
-        mbar_init(&bars->p_ready[x][y], 8);       // the 8 softmax warps of a tile
+        mbar_init(&bars->p_ready[x][y], 8);
         mbar_init(&bars->pv_done[x][y], 1);
       }
       mbar_init(&bars->o_free[x], 8);
@@ -235,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int u = atomicAdd(unit_counter, 1);
         if (u >= num_units) u = -1;
         const int slot = un & 1;
-        if (!mbar_wait(&bars->info_empty[slot], ((un >> 1) & 1) ^ 1)) { ok = false; break; }
+        if (!mbar_wait_sleep(&bars->info_empty[slot], ((un >> 1) & 1) ^ 1)) { ok = false; break; }
         UnitInfo U = {u, 0, 0, 0, 0, 0};
         if (u >= 0) U = unit_of(a, u);
         bars->info[slot] = U;
@@ -243,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u < 0 || aborted(bars)) break;
         const int32_t* klist =
             a.kept + (static_cast<int64_t>(U.b * a.Hkv + U.g) * a.nqb + U.i) * a.max_kept;
-        if (!mbar_wait(&bars->q_empty, (un & 1) ^ 1)) { ok = false; break; }
+        if (!mbar_wait_sleep(&bars->q_empty, (un & 1) ^ 1)) { ok = false; break; }
         mbar_arrive_expect_tx(&bars->q_full, ntiles * 2 * C::kHalves * 8192);
         for (int t = 0; t < ntiles; ++t)
           for (int hh = 0; hh < 2; ++hh) {
@@ -271,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (rk < 0) rk = 0;
           }
           const int s = kc % NS;
-          if (!mbar_wait(&bars->kv_empty[s], ((kc / NS) & 1) ^ 1)) { ok = false; break; }
+          if (!mbar_wait_sleep(&bars->kv_empty[s], ((kc / NS) & 1) ^ 1)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars->kv_full[s], C::kStage);
           unsigned char* st = smem + C::kOffKV + s * C::kStage;
           for (int x = 0; x < C::kHalves; ++x)
@@ -286,42 +297,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) set_abort(bars, a.status);
       // copies in flight must land before the CTA exits (bounded)
       for (uint32_t k = (kc > NS ? kc - NS : 0); k < kc; ++k)
-        mbar_wait(&bars->kv_full[k % NS], (k / NS) & 1, 100000000ull);
-      if (un > 0) mbar_wait(&bars->q_full, (un - 1) & 1, 100000000ull);
+        mbar_wait_sleep(&bars->kv_full[k % NS], (k / NS) & 1, 100000000ull);
+      if (un > 0) mbar_wait_sleep(&bars->q_full, (un - 1) & 1, 100000000ull);
     }
   } else if (warp == kWarpS0 || warp == kWarpS0 + 1) {
     // ------------------------------------------ score-MMA issuer of tile t
-    // S_t(j) = Q_t K_j^T into S buffer j % 2, once P_t(j-2).V (the last reader of
-    // that buffer) has completed; at most two steps ahead of the P.V issuer.
+    // S_t(j) = Q_t K_j^T into the S buffer of tile t, once the softmax warps have
+    // loaded S_t(j-1) from it.
     const int t = warp - kWarpS0;
     if (lane == 0) {
       const uint32_t idS = tc::idesc_f16(128, 64, 1, false);
       const uint32_t sbase = smem_u32(smem);
       const uint64_t dq = tc::smem_desc_sw128(sbase + t * C::kTile, 16, 1024);
-      const uint32_t s_tm = tmem + 256 + 128 * t;
+      const uint32_t s_tm = tmem + 256 + 64 * t;
       uint32_t un = 0, kc = 0;
       bool ok = true;
       while (ok) {
         const int slot = un & 1;
-        if (!mbar_wait(&bars->info_full[slot], (un >> 1) & 1)) { ok = false; break; }
+        if (!mbar_wait_sleep(&bars->info_full[slot], (un >> 1) & 1)) { ok = false; break; }
         const UnitInfo U = bars->info[slot];
         mbar_arrive(&bars->info_empty[slot]);
         if (U.u < 0 || aborted(bars)) break;
         if (t >= ntiles) { ++un; continue; }
         const int n = U.cnt > 0 ? U.cnt : 1;
-        if (!mbar_wait(&bars->q_full, un & 1)) { ok = false; break; }
+        if (!mbar_wait_sleep(&bars->q_full, un & 1)) { ok = false; break; }
         for (int jj = 0; jj < n; ++jj) {
           const uint32_t j = kc + jj;
           const int s = j % NS;
-          if (j >= 2 && !mbar_wait(&bars->pv_done[t][j & 1], ((j - 2) >> 1) & 1)) { ok = false; break; }
-          if (!mbar_wait(&bars->kv_full[s], (j / NS) & 1)) { ok = false; break; }
+          if (j >= 1 && !mbar_wait_sleep(&bars->s_free[t], (j - 1) & 1)) { ok = false; break; }
+          if (!mbar_wait_sleep(&bars->kv_full[s], (j / NS) & 1)) { ok = false; break; }
           tc::fence_after_sync();
           const uint64_t dk = tc::smem_desc_sw128(sbase + C::kOffKV + s * C::kStage, 16, 1024);
 #pragma unroll
           for (int ks = 0; ks < C::kKsteps; ++ks)
-            tc::mma_ss(s_tm + 64 * (j & 1), dq + (((ks >> 2) * C::kSlab + (ks & 3) * 32) >> 4),
+            tc::mma_ss(s_tm, dq + (((ks >> 2) * C::kSlab + (ks & 3) * 32) >> 4),
                        dk + (((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), idS, ks > 0);
-          tc::commit(&bars->s_full[t][j & 1]);
+          tc::commit(&bars->s_full[t]);
         }
         if (!ok) break;
         tc::commit(&bars->q_empty);   // Q of this tile is free once these MMAs complete
@@ -331,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) set_abort(bars, a.status);
       // every MMA this thread issued must finish before tensor memory is freed (bounded)
       tc::commit(&bars->mma_done[t]);
-      mbar_wait(&bars->mma_done[t], 0, 200000000ull);
+      mbar_wait_sleep(&bars->mma_done[t], 0, 200000000ull);
     }
   } else if (warp == kWarpPV) {
     // ------------------------------------------- P.V issuer of both tiles
@@ -345,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       while (ok) {
         const int slot = un & 1;
-        if (!mbar_wait(&bars->info_full[slot], (un >> 1) & 1)) { ok = false; break; }
+        if (!mbar_wait_sleep(&bars->info_full[slot], (un >> 1) & 1)) { ok = false; break; }
         const UnitInfo U = bars->info[slot];
         mbar_arrive(&bars->info_empty[slot]);
         if (U.u < 0 || aborted(bars)) break;
@@ -356,10 +367,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t dv =
               tc::smem_desc_sw128(sbase + C::kOffKV + s * C::kStage + C::kBlk, 8192, 1024);
           for (int t = 0; t < ntiles; ++t) {
-            if (jj == 0 && un > 0 && !mbar_wait(&bars->o_free[t], (un - 1) & 1)) { ok = false; break; }
-            if (!mbar_wait(&bars->p_ready[t][j & 1], (j >> 1) & 1)) { ok = false; break; }
+            if (jj == 0 && un > 0 && !mbar_wait_sleep(&bars->o_free[t], (un - 1) & 1)) { ok = false; break; }
+            if (!mbar_wait_sleep(&bars->p_ready[t][j & 1], (j >> 1) & 1)) { ok = false; break; }
             tc::fence_after_sync();
-            const uint32_t o_tm = tmem + 128 * t, p_tm = tmem + 256 + 128 * t + 64 * (j & 1);
+            const uint32_t o_tm = tmem + 128 * t, p_tm = tmem + 384 + 64 * t + 32 * (j & 1);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               tc::mma_ts(o_tm, p_tm + kk * 8, dv + ((kk * 2048) >> 4), idPV, jj > 0 || kk > 0);
@@ -373,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) set_abort(bars, a.status);
       tc::commit(&bars->mma_done[2]);
-      mbar_wait(&bars->mma_done[2], 0, 200000000ull);
+      mbar_wait_sleep(&bars->mma_done[2], 0, 200000000ull);
     }
   } else if (warp >= kWarpSm0 && warp < kWarpSm0 + 16) {
     // ----------------------------------------------------------- softmax warps
@@ -390,7 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rbase = q4 * 32 + hseg * 16;
     const int ra = rbase + t1, rb = ra + 8;
     const uint32_t lane_addr = static_cast<uint32_t>(rbase) << 16;
-    const uint32_t s_col0 = tmem + lane_addr + 256 + 128 * t;
+    const uint32_t s_col = tmem + lane_addr + 256 + 64 * t;
+    const uint32_t p_col0 = tmem + lane_addr + 384 + 64 * t;
     const uint32_t o_col = tmem + lane_addr + 128 * t;
     const float sc = a.scale_log2;
     const float2 sc2 = make_float2(sc, sc);
@@ -423,12 +435,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int jj = 0; jj < n; ++jj, ++kc) {
         const int blk_nx = jj + 1 < U.cnt ? klist[jj + 1] : U.i;
         const int buf = kc & 1;
-        if (!warp_wait(&bars->s_full[t][buf], (kc >> 1) & 1)) { ok = false; break; }
+        if (!warp_wait(&bars->s_full[t], kc & 1)) { ok = false; break; }
         tc::fence_after_sync();
-        const uint32_t s_col = s_col0 + 64 * buf;
         uint32_t sr[32];
         tc::ld16x256_x8(s_col, sr);
         tc::wait_ld();
+        // S is in registers: the score MMAs of the next step may overwrite it
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[t]);
         // masks: the causal diagonal block and blocks that failed validation
         if (mode != 0) {
           const int dblk = mode == 2 ? 0 : blk;
@@ -495,7 +510,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           sr[2 * k] = pack_f16(pa.x, pa.y);
           sr[2 * k + 1] = pack_f16(pb.x, pb.y);
         }
-        tc::st16x128_x8(s_col, *reinterpret_cast<const uint32_t(*)[16]>(&sr[0]));
+        // P buffer kc % 2 was last read by the P.V of step kc - 2
+        if (kc >= 2) {
+          const uint32_t jp = kc - 2;
+          if (!warp_wait(&bars->pv_done[t][jp & 1], (jp >> 1) & 1)) { ok = false; break; }
+          tc::fence_after_sync();
+        }
+        tc::st16x128_x8(p_col0 + 32 * buf, *reinterpret_cast<const uint32_t(*)[16]>(&sr[0]));
         if (any_up && jj > 0) {
           // rescale the O rows accumulated so far (warp-wide: tcgen05.ld/st are
           // collective), once the P.V of the previous step has completed

@@ -22,6 +22,12 @@ namespace bsa {
 namespace {
 
 constexpr int kWarps = 4;
+
+BSA_DEVFN float max3f(float x, float y, float z) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(x), "f"(y), "f"(z));
+  return r;
+}
 constexpr int kBatch = 32;  // key blocks per shared-memory combine
 
 template <int HP>  // head pairs = ceil(G / 2)
@@ -38,6 +44,7 @@ __global__ void __launch_bounds__(kWarps * 32) score_prefill_kernel(const ScoreP
   // query fragments: tq group tg (8 tokens), head pair hp
   uint32_t aq[2][HP][4];
   float w[HP][2];
+  float2 w0p[HP], w1p[HP];   // the weights of the pair's two heads, duplicated for FFMA2
   const char* qbase = static_cast<const char*>(a.q_idx);
   const float dflt = 1.0f / static_cast<float>(a.G);
 #pragma unroll
@@ -61,6 +68,11 @@ __global__ void __launch_bounds__(kWarps * 32) score_prefill_kernel(const ScoreP
       aq[tg][hp][2] = x0.y;
       aq[tg][hp][3] = x1.y;
     }
+  }
+#pragma unroll
+  for (int hp = 0; hp < HP; ++hp) {
+    w0p[hp] = make_float2(w[hp][0], w[hp][0]);
+    w1p[hp] = make_float2(w[hp][1], w[hp][1]);
   }
   // query tokens of this lane that exist (a ragged last query block)
   const bool q0v = i * kBlock + 16 * warp + gid < a.T;
@@ -90,18 +102,17 @@ __global__ void __launch_bounds__(kWarps * 32) score_prefill_kernel(const ScoreP
           const uint2 kv = *reinterpret_cast<const uint2*>(kb + (nt * 8 + gid) * 32 + tig * 8);
 #pragma unroll
           for (int tg = 0; tg < 2; ++tg) {
-            float u0 = 0.f, u1 = 0.f;
+            // u = (key 2*tig, key 2*tig + 1): two-wide FMAs, head by head in order
+            float2 u = make_float2(0.f, 0.f);
 #pragma unroll
             for (int hp = 0; hp < HP; ++hp) {
               float c[4] = {0.f, 0.f, 0.f, 0.f};
               mma_bf16(c, aq[tg][hp], kv.x, kv.y);
-              u0 = fmaf(w[hp][0], fmaxf(c[0], 0.f), u0);
-              u0 = fmaf(w[hp][1], fmaxf(c[2], 0.f), u0);
-              u1 = fmaf(w[hp][0], fmaxf(c[1], 0.f), u1);
-              u1 = fmaf(w[hp][1], fmaxf(c[3], 0.f), u1);
+              u = __ffma2_rn(w0p[hp], make_float2(fmaxf(c[0], 0.f), fmaxf(c[1], 0.f)), u);
+              u = __ffma2_rn(w1p[hp], make_float2(fmaxf(c[2], 0.f), fmaxf(c[3], 0.f)), u);
             }
             const bool qv = tg == 0 ? q0v : q1v;
-            if (qv) mx = fmaxf(mx, fmaxf(u0, u1));
+            if (qv) mx = max3f(mx, u.x, u.y);
           }
         }
 #pragma unroll
