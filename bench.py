@@ -159,13 +159,18 @@ def barrier(world):
 
 
 # ---------------------------------------------------------------- byte / FLOP accounting
-def decode_bytes(w, kept_count, seq_lens):
-    """Algorithmic bytes of one decode step and of its attention call."""
+def decode_bytes(w, kept_count, seq_lens, index_cache="bf16"):
+    """Algorithmic bytes of one decode step and of its attention call. Index keys:
+    32 B per token in bf16; a 576-byte record per visible 64-token block (9 B per
+    token) in the 4-bit formats."""
     B, Hq, Hkv, d, r = w.B, w.Hq, w.Hkv, w.d, w.r
     kc = kept_count.to(torch.int64).cpu()
     lens = seq_lens.to(torch.int64).cpu()
     kv = int(kc.sum()) * 64 * d * 2 * 2                 # K and V of every kept block
-    idx = int(lens.sum()) * Hkv * r * 2                 # every index key
+    if index_cache == "bf16":
+        idx = int(lens.sum()) * Hkv * r * 2             # every index key
+    else:
+        idx = int(((lens + 63) // 64).sum()) * Hkv * 576 + 4
     q = B * Hq * d * 2
     q_idx = B * Hq * r * 2
     o = B * Hq * d * 2 + B * Hq * 4                     # bf16 output + fp32 lse
@@ -205,6 +210,13 @@ def run_ours(args, world, rank, local):
         dprob = bsa.problem_for(wd, seq_lens=xd["seq_lens"], head_w=xd["head_w"])
         dstep = bsa.DecodeStep(dprob, device=dev, keep_f32=False)
         k_idx_c, K_c, V_c = bsa.caches_for(xd)
+        if args.index_cache != "bf16":
+            # the selector cache is quantised once, as when the keys are written
+            fmt = bsa.IDX_FP4 if args.index_cache == "fp4" else bsa.IDX_INT4
+            qc = bsa.contiguous_qcache(wd.B, wd.Hkv, wd.T, fmt, device=dev)
+            bsa.bsa_quantize_index_keys(dprob, k_idx_c, qc, dstep.status)
+            k_idx_c = qc
+            torch.cuda.synchronize()
     if do_pf:
         xp = W.make_prefill_inputs(wp, dev)
         pprob = bsa.problem_for(wp, head_w=xp["head_w"])
@@ -219,7 +231,10 @@ def run_ours(args, world, rank, local):
         if ev:
             ev["d0"].record(stream)
         if do_dec:
-            bsa.bsa_score_blocks(dprob, xd["q_idx"], k_idx_c, dstep.scores, dstep.status)
+            if isinstance(k_idx_c, bsa.QCache):
+                bsa.bsa_score_blocks_q(dprob, xd["q_idx"], k_idx_c, dstep.scores, dstep.status)
+            else:
+                bsa.bsa_score_blocks(dprob, xd["q_idx"], k_idx_c, dstep.scores, dstep.status)
             bsa.bsa_select_top_p(dprob, dstep.scores, dstep.kept, dstep.kept_count, dstep.status)
         if ev:
             ev["a0"].record(stream)
@@ -281,7 +296,7 @@ def run_ours(args, world, rank, local):
     dec = pre = None
     roof_dec = roof_pf = None
     if do_dec:
-        by = decode_bytes(wd, dstep.kept_count, xd["seq_lens"])
+        by = decode_bytes(wd, dstep.kept_count, xd["seq_lens"], args.index_cache)
         dec_sum, att_avg, dec_avg = max(dec_sum, 1e-9), max(att_avg, 1e-9), max(dec_avg, 1e-9)
         tokens_per_s = world * wd.B * args.steps / (dec_sum / 1e3)
         attn_gbs = by["attention"] / (att_avg / 1e3) / 1e9
@@ -316,13 +331,14 @@ def run_ours(args, world, rank, local):
            run_e2e(args, dprob, dstep, xd, k_idx_c, K_c, V_c, stream, world))
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and do_dec:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and do_dec and args.index_cache == "bf16":
         cpu = cpu_baseline_decode(wd, xd, dstep, budget_s=args.cpu_budget)
 
     clocks = clk.summary()
     config = {"workload": " + ".join(w.name for w, on in ((wd, do_dec), (wp, do_pf)) if on)}
     if do_dec:
         config["decode"] = describe(wd)
+        config["index_cache"] = args.index_cache
     if do_pf:
         config["prefill"] = describe(wp)
     config["l2"] = ("decode inputs exceed L2; a 256 MB buffer is written before each prefill")
@@ -486,6 +502,9 @@ def main():
     ap.add_argument("--prefill-workload", default=PREFILL_WL, choices=sorted(
         k for k, v in W.WORKLOADS.items() if v.phase == "prefill"))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--index-cache", choices=["bf16", "fp4", "int4"], default="bf16",
+                    help="decode index-key cache: bf16 (the method as configured) or the "
+                         "4-bit microscaled selector cache")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

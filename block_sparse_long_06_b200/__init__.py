@@ -28,8 +28,10 @@ BLOCK = 64
 
 EXPORTED = ["bsa_max_kept", "bsa_workspace_size", "bsa_score_blocks", "bsa_select_top_p",
             "bsa_decode", "bsa_prefill", "bsa_status_string", "bsa_last_cuda_error",
-            "bsa_decode_noalloc"]
+            "bsa_decode_noalloc", "bsa_quantize_index_keys", "bsa_score_blocks_q"]
 NOALLOC_SCRATCH_BYTES = 8 << 20
+IDX_FP4, IDX_INT4 = 1, 2
+QIDX_RECORD_BYTES = 576
 
 
 class BsaError(RuntimeError):
@@ -41,6 +43,14 @@ class CCache(ctypes.Structure):
                 ("block_stride", ctypes.c_int64), ("head_stride", ctypes.c_int64),
                 ("page_table", ctypes.c_void_p), ("page_table_stride", ctypes.c_int32),
                 ("num_pages", ctypes.c_int32), ("extent", ctypes.c_int64)]
+
+
+class CQCache(ctypes.Structure):
+    _fields_ = [("records", ctypes.c_void_p), ("gscale", ctypes.c_void_p),
+                ("seq_stride", ctypes.c_int64), ("block_stride", ctypes.c_int64),
+                ("head_stride", ctypes.c_int64), ("page_table", ctypes.c_void_p),
+                ("page_table_stride", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("extent", ctypes.c_int64), ("format", ctypes.c_int32)]
 
 
 class CProblem(ctypes.Structure):
@@ -80,6 +90,10 @@ def load_library(path: str = LIB_PATH):
         f.restype = ctypes.c_int
     lib.bsa_decode_noalloc.argtypes = [P, vp, CCache, CCache, vp, vp, vp, vp, vp, vp, vp]
     lib.bsa_decode_noalloc.restype = ctypes.c_int
+    lib.bsa_quantize_index_keys.argtypes = [P, CCache, CQCache, vp, vp]
+    lib.bsa_quantize_index_keys.restype = ctypes.c_int
+    lib.bsa_score_blocks_q.argtypes = [P, vp, CQCache, vp, vp, vp]
+    lib.bsa_score_blocks_q.restype = ctypes.c_int
     lib.bsa_status_string.argtypes = [ctypes.c_int]
     lib.bsa_status_string.restype = ctypes.c_char_p
     lib.bsa_last_cuda_error.argtypes = []
@@ -175,6 +189,43 @@ def paged_cache(pool: torch.Tensor, page_table: torch.Tensor) -> Cache:
     return Cache(pool, 0, H * BLOCK * w, BLOCK * w, page_table, P)
 
 
+@dataclass
+class QCache:
+    """A 4-bit index-key cache (bsa_qcache_t): 576-byte records of 64 tokens, plus
+    the cache scale. `records` is a uint8 tensor, `gscale` a float32 [1] tensor."""
+    records: torch.Tensor
+    gscale: torch.Tensor
+    fmt: int
+    seq_stride: int
+    block_stride: int
+    head_stride: int
+    page_table: Optional[torch.Tensor] = None
+    num_pages: int = 0
+
+    def c(self) -> CQCache:
+        pt = self.page_table
+        return CQCache(self.records.data_ptr(), self.gscale.data_ptr(), self.seq_stride,
+                       self.block_stride, self.head_stride, None if pt is None else pt.data_ptr(),
+                       0 if pt is None else pt.shape[1], self.num_pages,
+                       self.records.numel() // QIDX_RECORD_BYTES, self.fmt)
+
+
+def contiguous_qcache(B: int, Hkv: int, T: int, fmt: int, device=None) -> QCache:
+    """Zeroed [B, Hkv, nb] records (nb = ceil(T/64))."""
+    nb = (T + BLOCK - 1) // BLOCK
+    rec = torch.zeros(B * Hkv * nb * QIDX_RECORD_BYTES, dtype=torch.uint8, device=device)
+    gs = torch.zeros(1, dtype=torch.float32, device=device)
+    return QCache(rec, gs, fmt, Hkv * nb, 1, nb)
+
+
+def paged_qcache(num_pages: int, Hkv: int, page_table: torch.Tensor, fmt: int, device=None) -> QCache:
+    """Zeroed [P, Hkv] records addressed through a [B, nb] int32 page table."""
+    assert page_table.dtype == torch.int32 and page_table.is_contiguous()
+    rec = torch.zeros(num_pages * Hkv * QIDX_RECORD_BYTES, dtype=torch.uint8, device=device)
+    gs = torch.zeros(1, dtype=torch.float32, device=device)
+    return QCache(rec, gs, fmt, 0, Hkv, 1, page_table, num_pages)
+
+
 # ------------------------------------------------------------------ the C entry points
 def bsa_max_kept(prob: Problem) -> int:
     return load_library().bsa_max_kept(ctypes.byref(prob.c()))
@@ -192,6 +243,20 @@ def bsa_score_blocks(prob: Problem, q_idx, k_idx: Cache, block_scores, dev_statu
     _check(load_library().bsa_score_blocks(ctypes.byref(prob.c()), _ptr(q_idx), k_idx.c(),
                                            _ptr(block_scores), _ptr(dev_status), _stream(stream)),
            "bsa_score_blocks")
+
+
+def bsa_quantize_index_keys(prob: Problem, k_idx: Cache, out: QCache, dev_status=None,
+                            stream=None):
+    _check(load_library().bsa_quantize_index_keys(ctypes.byref(prob.c()), k_idx.c(), out.c(),
+                                                  _ptr(dev_status), _stream(stream)),
+           "bsa_quantize_index_keys")
+
+
+def bsa_score_blocks_q(prob: Problem, q_idx, k_idx: QCache, block_scores, dev_status=None,
+                       stream=None):
+    _check(load_library().bsa_score_blocks_q(ctypes.byref(prob.c()), _ptr(q_idx), k_idx.c(),
+                                             _ptr(block_scores), _ptr(dev_status), _stream(stream)),
+           "bsa_score_blocks_q")
 
 
 def bsa_select_top_p(prob: Problem, block_scores, kept, kept_count, dev_status=None, stream=None):
@@ -256,9 +321,13 @@ class DecodeStep:
         self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def run(self, q, q_idx, k_idx: Cache, k: Cache, v: Cache, stream=None):
+    def run(self, q, q_idx, k_idx, k: Cache, v: Cache, stream=None):
+        """k_idx: a bf16 index-key Cache or a 4-bit QCache."""
         p = self.prob
-        bsa_score_blocks(p, q_idx, k_idx, self.scores, self.status, stream)
+        if isinstance(k_idx, QCache):
+            bsa_score_blocks_q(p, q_idx, k_idx, self.scores, self.status, stream)
+        else:
+            bsa_score_blocks(p, q_idx, k_idx, self.scores, self.status, stream)
         bsa_select_top_p(p, self.scores, self.kept, self.kept_count, self.status, stream)
         bsa_decode(p, q, k, v, self.kept, self.kept_count, self.o, self.lse, self.o_f32,
                    self.workspace, self.status, stream)
@@ -316,7 +385,7 @@ def caches_for(inputs: dict):
     return k_idx, contiguous_cache(inputs["K"]), contiguous_cache(inputs["V"])
 
 
-def decode_step_host(step: DecodeStep, q_host, q_idx_host, k_idx: Cache, k: Cache, v: Cache,
+def decode_step_host(step: DecodeStep, q_host, q_idx_host, k_idx, k: Cache, v: Cache,
                      o_host, lse_host, q_dev=None, q_idx_dev=None, stream=None):
     """One decode step from host buffers: copy the new query (q, q_idx; pinned host
     tensors) to the device, run score -> select -> attend, copy o and lse back into

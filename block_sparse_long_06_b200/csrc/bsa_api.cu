@@ -149,6 +149,32 @@ DecodePlan decode_plan(const bsa_problem_t* p, int num_sms) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// 4-bit index-key cache checks: 16-byte aligned records, record strides >= 0,
+// a valid format and a scale pointer.
+bsa_status_t check_qcache(const bsa_qcache_t& c, const bsa_problem_t* p) {
+  if (c.records == nullptr || !aligned16(c.records) || c.gscale == nullptr || c.extent <= 0)
+    return BSA_ERR_INVALID_ARG;
+  if (c.format != BSA_IDX_FP4 && c.format != BSA_IDX_INT4) return BSA_ERR_INVALID_ARG;
+  if (c.seq_stride < 0 || c.block_stride <= 0 || c.head_stride < 0) return BSA_ERR_INVALID_ARG;
+  if (c.page_table != nullptr) {
+    if (c.num_pages <= 0 || c.page_table_stride < nblocks(p->T)) return BSA_ERR_INVALID_ARG;
+  }
+  return BSA_OK;
+}
+
+bsa::CacheView qview(const bsa_qcache_t& c) {
+  bsa::CacheView v;
+  v.base = c.records;
+  v.seq_stride = c.seq_stride;
+  v.block_stride = c.block_stride;
+  v.head_stride = c.head_stride;
+  v.page_table = c.page_table;
+  v.pt_stride = c.page_table_stride;
+  v.num_pages = c.num_pages;
+  v.extent = c.extent;
+  return v;
+}
+
 }  // namespace
 
 namespace bsa {
@@ -234,6 +260,58 @@ bsa_status_t bsa_score_blocks(const bsa_problem_t* p, const void* q_idx, bsa_cac
     a.idx_scale = idx_scale_of(p);
     e = bsa::launch_score_prefill(a, num_sms, s);
   }
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e);
+}
+
+bsa_status_t bsa_quantize_index_keys(const bsa_problem_t* p, bsa_cache_t k_idx, bsa_qcache_t out,
+                                     int32_t* dev_status, void* stream) {
+  bsa_status_t st = check_problem(p);
+  if (st != BSA_OK) return st;
+  if (p->phase != BSA_PHASE_DECODE) return BSA_ERR_UNSUPPORTED;
+  if ((st = check_cache(k_idx, p, p->r, false)) != BSA_OK) return st;
+  if ((st = check_qcache(out, p)) != BSA_OK) return st;
+  bsa::QuantArgs a{};
+  a.src = view(k_idx);
+  a.dst = qview(out);
+  a.gscale = out.gscale;
+  a.seq_lens = p->seq_lens;
+  a.status = dev_status;
+  a.B = p->B;
+  a.Hkv = p->Hkv;
+  a.T = p->T;
+  a.nb = nblocks(p->T);
+  a.fmt = out.format;
+  const cudaError_t e = bsa::launch_quantize_index(a, num_sms_current(), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e);
+}
+
+bsa_status_t bsa_score_blocks_q(const bsa_problem_t* p, const void* q_idx, bsa_qcache_t k_idx,
+                                float* block_scores, int32_t* dev_status, void* stream) {
+  bsa_status_t st = check_problem(p);
+  if (st != BSA_OK) return st;
+  if (p->phase != BSA_PHASE_DECODE) return BSA_ERR_UNSUPPORTED;
+  if (q_idx == nullptr || block_scores == nullptr || !aligned16(q_idx)) return BSA_ERR_INVALID_ARG;
+  if ((st = check_qcache(k_idx, p)) != BSA_OK) return st;
+  bsa::ScoreDecodeArgs a{};
+  a.q_idx = q_idx;
+  a.kidx = qview(k_idx);
+  a.seq_lens = p->seq_lens;
+  a.head_w = p->head_w;
+  a.scores = block_scores;
+  a.status = dev_status;
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = p->Hq / p->Hkv;
+  a.T = p->T;
+  a.nb_max = nblocks(p->T);
+  const int cb = bsa::score_decode_chunk_blocks();
+  a.chunks_per_row = (a.nb_max + cb - 1) / cb;
+  a.total_items = static_cast<int64_t>(p->B) * p->Hkv * a.chunks_per_row;
+  a.idx_scale = idx_scale_of(p);
+  a.kfmt = k_idx.format;
+  a.gscale = k_idx.gscale;
+  const cudaError_t e = bsa::launch_score_decode(a, num_sms_current(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e);
 }
 

@@ -186,6 +186,14 @@ BSA_DEVFN float2 unpack_bf16(uint32_t x) {
 }
 
 // Hardware base-2 exponential (MUFU), approximate, flush-to-zero.
+// Value of an E4M3 (FP8, bias 7, with subnormals) code; 0x7F (NaN) is never produced
+// by the index-key quantiser.
+BSA_DEVFN float e4m3_value(uint32_t code) {
+  const uint32_t e = (code >> 3) & 15u, m = code & 7u;
+  if (e == 0u) return __fmul_rn(static_cast<float>(m), 0.001953125f);   // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
 BSA_DEVFN float ex2(float x) {
   float y;
   asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

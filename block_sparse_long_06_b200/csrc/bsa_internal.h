@@ -28,6 +28,20 @@ struct ScoreDecodeArgs {
   int B, Hq, Hkv, G, T, nb_max, chunks_per_row;
   int64_t total_items;
   float idx_scale;
+  int kfmt;                   // 0: bf16 keys; 1: FP4 / 2: INT4 records (kidx counts records)
+  const float* gscale;        // 4-bit formats: the cache scale g (device)
+};
+
+// 4-bit index-key cache: 576-byte records of 64 tokens (codes, then scales).
+constexpr int kQRecord = 576;
+
+struct QuantArgs {
+  CacheView src;              // bf16 index keys, width 16
+  CacheView dst;              // records; strides and extent count records
+  float* gscale;              // one float: amax scratch, then g
+  const int32_t* seq_lens;    // [B] or null
+  int32_t* status;
+  int B, Hkv, T, nb, fmt;     // fmt 1 = FP4, 2 = INT4
 };
 
 struct ScorePrefillArgs {
@@ -83,6 +97,7 @@ struct PrefillArgs {
 
 // Each launcher returns the cudaError_t of its launch.
 cudaError_t launch_score_decode(const ScoreDecodeArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_quantize_index(const QuantArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_score_prefill(const ScorePrefillArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,

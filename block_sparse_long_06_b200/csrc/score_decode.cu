@@ -21,6 +21,13 @@
 //  * epilogue in fp32: ReLU, head weights, head sum with two shuffles (each lane
 //    pair exchanges the half it does not keep), running max, a 4-shuffle warp max
 //    per block, then the stage is released through its "empty" mbarrier.
+//  * 4-bit index keys (SpotAttention, Methodology §4; format in include/bsa.h):
+//    the same kernel streams 576-byte block records (9 B per token), with four
+//    CTAs per SM since the unpacking makes it latency- rather than HBM-bound. A lane turns its token's four 4-bit codes into
+//    bf16 with two byte-permute table lookups plus the sign bits (every code value
+//    is exact in bf16), runs the same MMA on the unscaled codes, and multiplies
+//    the token's ReLU head sum by its E4M3 scale (ReLU is positively homogeneous,
+//    and the scales are > 0); the cache scale g multiplies the block score.
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
 
@@ -29,11 +36,7 @@ namespace {
 
 constexpr int kConsumers = 8;                              // consumer warps = blocks per chunk
 constexpr int kChunk = kConsumers;                         // blocks per item / stage
-constexpr int kStages = 6;
-constexpr int kBlockBytes = kBlock * kR * 2;               // 2048
-constexpr int kStageBytes = kChunk * kBlockBytes;          // 16 KB
 constexpr int kThreads = (kConsumers + 1) * 32;
-constexpr int kCtasPerSm = 2;
 
 struct StageInfo {
   int row;        // b * Hkv + g
@@ -42,11 +45,50 @@ struct StageInfo {
   uint32_t ok;    // bit q: block j0 + q was copied
 };
 
+// KF: key format, 0 = bf16 rows (32 B per token), 1 = FP4 / 2 = INT4 records.
+template <int KF>
 struct ScoreSmem {
+  static constexpr int kBlockBytes = KF == 0 ? kBlock * kR * 2 : kQRecord;   // 2048 or 576
+  static constexpr int kStages = KF == 0 ? 6 : 8;
+  // 4-bit keys cost more instructions per byte: more resident CTAs hide the latency
+  static constexpr int kCtasPerSm = KF == 0 ? 2 : 4;
+  static constexpr int kStageBytes = kChunk * kBlockBytes;
   static constexpr int kRing = kStages * kStageBytes;
   static constexpr int kInfo = kStages * static_cast<int>(sizeof(StageInfo));
   static constexpr int kTotal = kRing + kInfo + 2 * kStages * 8 + 128;
 };
+
+// Record index of block `blk` of (b, g) in a 4-bit cache, false when invalid.
+BSA_DEVFN bool block_record(const CacheView& c, int b, int g, int blk, int64_t& rec) {
+  int64_t phys = blk;
+  if (c.page_table != nullptr) {
+    phys = c.page_table[static_cast<int64_t>(b) * c.pt_stride + blk];
+    if (phys < 0 || phys >= c.num_pages) return false;
+  }
+  rec = static_cast<int64_t>(b) * c.seq_stride + phys * c.block_stride +
+        static_cast<int64_t>(g) * c.head_stride;
+  return rec >= 0 && rec + 1 <= c.extent;
+}
+
+// Four 4-bit codes (elements 4t..4t+3 of a token, low nibble first) -> four bf16
+// values (two bf16x2 words). Byte-permute tables give the low and high byte of
+// the bf16 of each magnitude index; the sign bits are ORed in.
+template <int KF>
+BSA_DEVFN uint2 dequant4(uint32_t c16) {
+  // magnitudes: FP4 (E2M1) 0, .5, 1, 1.5, 2, 3, 4, 6; INT4 0..7
+  constexpr uint32_t kLoX = KF == 1 ? 0xC0800000u : 0x40008000u;
+  constexpr uint32_t kLoY = KF == 1 ? 0xC0804000u : 0xE0C0A080u;
+  constexpr uint32_t kHiX = KF == 1 ? 0x3F3F3F00u : 0x40403F00u;
+  constexpr uint32_t kHiY = 0x40404040u;
+  const uint32_t sel = c16 & 0x7777u;
+  const uint32_t lo = __byte_perm(kLoX, kLoY, sel), hi = __byte_perm(kHiX, kHiY, sel);
+  // sign bits 3, 7 (11, 15) of the codes -> bits 15, 31 of the words: one multiply
+  // places both copies (x * (2^12 + 2^24) puts bit 3 at 15 and bit 7 at 31).
+  const uint32_t s0 = (c16 & 0x88u) * 0x01001000u, s1 = (c16 & 0x8800u) * 0x00010010u;
+  const uint32_t w0 = __byte_perm(lo, hi, 0x5140u) | (s0 & 0x80008000u);
+  const uint32_t w1 = __byte_perm(lo, hi, 0x7362u) | (s1 & 0x80008000u);
+  return make_uint2(w0, w1);
+}
 
 BSA_DEVFN int clamp_len(const ScoreDecodeArgs& a, int b) {
   int Tb = a.seq_lens ? a.seq_lens[b] : a.T;
@@ -66,17 +108,21 @@ BSA_DEVFN bool block_offset(const CacheView& c, int b, int g, int blk, int rows,
   return off >= 0 && off + static_cast<int64_t>(rows) * kR <= c.extent;
 }
 
-template <int NT>
+template <int NT, int KF>
 __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecodeArgs a) {
+  using SM = ScoreSmem<KF>;
+  constexpr int kStages = SM::kStages, kStageBytes = SM::kStageBytes, kBlockBytes = SM::kBlockBytes;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
   unsigned char* ring = smem;
-  StageInfo* info = reinterpret_cast<StageInfo*>(smem + ScoreSmem::kRing);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + ScoreSmem::kRing + ScoreSmem::kInfo);
+  StageInfo* info = reinterpret_cast<StageInfo*>(smem + SM::kRing);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kRing + SM::kInfo);
   uint64_t* empty = full + kStages;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ float scale_lut[128];   // E4M3 code -> value (4-bit keys)
+  if (KF != 0 && threadIdx.x < 128) scale_lut[threadIdx.x] = e4m3_value(threadIdx.x);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -95,7 +141,8 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       const char* kbase = static_cast<const char*>(a.kidx.base);
-      const bool contiguous = a.kidx.page_table == nullptr && a.kidx.block_stride == kBlock * kR;
+      const bool contiguous =
+          a.kidx.page_table == nullptr && a.kidx.block_stride == (KF == 0 ? kBlock * kR : 1);
       // walk the item range incrementally: (row, j0) without a division per item
       int row = static_cast<int>(it0 / a.chunks_per_row);
       int j0 = static_cast<int>(it0 - static_cast<int64_t>(row) * a.chunks_per_row) * kChunk;
@@ -111,7 +158,29 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
         const int nblk = max(0, min(kChunk, nb_row - j0));      // blocks of the chunk that exist
         unsigned char* dst = ring + s * kStageBytes;
         uint32_t ok = 0, bytes = 0;
-        if (contiguous && nblk > 0) {
+        if (KF != 0 && contiguous && nblk > 0) {
+          // adjacent whole records: one range check, one copy
+          int64_t rec;
+          if (block_record(a.kidx, b, g, j0, rec) && rec + nblk <= a.kidx.extent) {
+            ok = (1u << nblk) - 1u;
+            bytes = nblk * kBlockBytes;
+          }
+          info[s] = StageInfo{row, j0, Tb, ok};
+          mbar_arrive_expect_tx(&full[s], bytes);
+          if (ok) bulk_g2s(dst, kbase + rec * kBlockBytes, bytes, &full[s]);
+        } else if (KF != 0) {
+          int64_t recs[kChunk];
+          for (int q = 0; q < nblk; ++q)
+            if (block_record(a.kidx, b, g, j0 + q, recs[q])) {
+              ok |= 1u << q;
+              bytes += kBlockBytes;
+            }
+          info[s] = StageInfo{row, j0, Tb, ok};
+          mbar_arrive_expect_tx(&full[s], bytes);
+          for (int q = 0; q < nblk; ++q)
+            if (ok & (1u << q))
+              bulk_g2s(dst + q * kBlockBytes, kbase + recs[q] * kBlockBytes, kBlockBytes, &full[s]);
+        } else if (contiguous && nblk > 0) {
           // the chunk's blocks are adjacent: one range check, one copy
           const int rows = min(nblk * kBlock, Tb - j0 * kBlock);
           int64_t off;
@@ -159,6 +228,7 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
 
   // ------------------------------------------------------------------ consumers
   const int gid = lane >> 2, tig = lane & 3;
+  const float kscale = KF == 0 ? 1.0f : *a.gscale;   // cache scale g of 4-bit keys
   int cur_row = -1;
   uint32_t bq[NT][2];
   float w0[NT], w1[NT];
@@ -186,8 +256,9 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
           bq[nt][1] = v.y;
         }
         const int h0 = nt * 8 + 2 * tig, h1 = h0 + 1;
-        w0[nt] = h0 < a.G ? (a.head_w ? a.head_w[g * a.G + h0] : dflt) : 0.f;
-        w1[nt] = h1 < a.G ? (a.head_w ? a.head_w[g * a.G + h1] : dflt) : 0.f;
+        // half weights: (w/2) * (c + |c|) = w * ReLU(c) exactly (c + |c| is 2c or +0)
+        w0[nt] = 0.5f * (h0 < a.G ? (a.head_w ? a.head_w[g * a.G + h0] : dflt) : 0.f);
+        w1[nt] = 0.5f * (h1 < a.G ? (a.head_w ? a.head_w[g * a.G + h1] : dflt) : 0.f);
       }
     }
     if (j < a.nb_max) {
@@ -207,18 +278,25 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
           const int r0 = mt * 16 + gid, r1 = r0 + 8;
-          const uint2 x0 = *reinterpret_cast<const uint2*>(blk + r0 * 32 + tig * 8);
-          const uint2 x1 = *reinterpret_cast<const uint2*>(blk + r1 * 32 + tig * 8);
+          uint2 x0, x1;
+          if constexpr (KF == 0) {
+            x0 = *reinterpret_cast<const uint2*>(blk + r0 * 32 + tig * 8);
+            x1 = *reinterpret_cast<const uint2*>(blk + r1 * 32 + tig * 8);
+          } else {
+            x0 = dequant4<KF>(*reinterpret_cast<const uint16_t*>(blk + r0 * 8 + tig * 2));
+            x1 = dequant4<KF>(*reinterpret_cast<const uint16_t*>(blk + r1 * 8 + tig * 2));
+          }
           const uint32_t af[4] = {x0.x, x1.x, x0.y, x1.y};
           float vr0 = 0.f, vr1 = 0.f;
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             float c[4] = {0.f, 0.f, 0.f, 0.f};
             mma_bf16(c, af, bq[nt][0], bq[nt][1]);
-            vr0 = fmaf(w0[nt], fmaxf(c[0], 0.f), vr0);
-            vr0 = fmaf(w1[nt], fmaxf(c[1], 0.f), vr0);
-            vr1 = fmaf(w0[nt], fmaxf(c[2], 0.f), vr1);
-            vr1 = fmaf(w1[nt], fmaxf(c[3], 0.f), vr1);
+            // ReLU on the FMA pipe (the ALU pipe is the busier one)
+            vr0 = fmaf(w0[nt], c[0] + fabsf(c[0]), vr0);
+            vr0 = fmaf(w1[nt], c[1] + fabsf(c[1]), vr0);
+            vr1 = fmaf(w0[nt], c[2] + fabsf(c[2]), vr1);
+            vr1 = fmaf(w1[nt], c[3] + fabsf(c[3]), vr1);
           }
           // head sum over the 4 lanes of a row group: even lanes keep token r0,
           // odd lanes token r1
@@ -227,6 +305,7 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
           keep += __shfl_xor_sync(0xffffffffu, send, 1);
           keep += __shfl_xor_sync(0xffffffffu, keep, 2);
           const int tok = odd ? r1 : r0;
+          if constexpr (KF != 0) keep *= scale_lut[blk[kBlock * 8 + tok] & 0x7Fu];   // token scale
           if (tok < valid) mx = fmaxf(mx, keep);
         }
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -234,7 +313,7 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         if (lane == 0) {
-          const float sc = a.idx_scale * mx;
+          const float sc = a.idx_scale * (kscale * mx);
           *out = sc;
           if (!isfinite(sc)) report(a.status, BSA_DEV_NONFINITE);
         }
@@ -245,18 +324,28 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
   }
 }
 
-}  // namespace
-
-cudaError_t launch_score_decode(const ScoreDecodeArgs& a, int num_sms, cudaStream_t s) {
-  if (a.total_items <= 0) return cudaSuccess;
-  const int smem = ScoreSmem::kTotal;
-  int64_t ctas = static_cast<int64_t>(num_sms) * kCtasPerSm;
+template <int KF>
+cudaError_t launch_fmt(const ScoreDecodeArgs& a, int num_sms, cudaStream_t s) {
+  const int smem = ScoreSmem<KF>::kTotal;
+  int64_t ctas = static_cast<int64_t>(num_sms) * ScoreSmem<KF>::kCtasPerSm;
   if (ctas > a.total_items) ctas = a.total_items;
-  auto kern = (a.G > 8) ? score_decode_kernel<2> : score_decode_kernel<1>;
+  auto kern = (a.G > 8) ? score_decode_kernel<2, KF> : score_decode_kernel<1, KF>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<static_cast<unsigned>(ctas), kThreads, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_score_decode(const ScoreDecodeArgs& a, int num_sms, cudaStream_t s) {
+  if (a.total_items <= 0) return cudaSuccess;
+  switch (a.kfmt) {
+    case 0: return launch_fmt<0>(a, num_sms, s);
+    case 1: return launch_fmt<1>(a, num_sms, s);
+    case 2: return launch_fmt<2>(a, num_sms, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 int score_decode_chunk_blocks() { return kChunk; }

@@ -150,6 +150,68 @@ bsa_status_t bsa_prefill(const bsa_problem_t* prob, const void* q, bsa_cache_t k
                          float* o_f32, void* workspace, size_t workspace_bytes,
                          int32_t* dev_status, void* stream);
 
+/* ------------------------------------------------------------------------
+ * 4-bit index-key cache (SpotAttention, Methodology §4: the selector's K cache
+ * may be stored as microscaled INT4 or FP4, about 3.5x smaller than bf16; the
+ * backbone's K/V cache is untouched).
+ *
+ * Format. Each token's r = 16 index-key elements are 16 4-bit codes plus one
+ * E4M3 (FP8) scale byte: 9 bytes instead of 32. A code is sign-magnitude: bit 3
+ * = sign, bits 0-2 = magnitude index m. FP4: magnitude = E2M1 value of m
+ * (0, 0.5, 1, 1.5, 2, 3, 4, 6); INT4: magnitude = m (0..7). One fp32 scale g
+ * covers the whole cache. Element c of a token is
+ *     k[c] = +-magnitude(m_c) * e4m3(scale) * g.
+ * Storage is one 576-byte record per (sequence, kv head, 64-token block): 64
+ * tokens x 8 bytes of codes (byte c holds element 2c in its low nibble and
+ * element 2c+1 in its high nibble), then the 64 scale bytes. Tokens t >= T_b of
+ * a partial last block hold zero codes and a zero scale.
+ *
+ * Addressing counts RECORDS: the record of block j of sequence b, kv head g is
+ *     records + 576 * (b*seq_stride + phys*block_stride + g*head_stride)
+ * with phys = page_table[b*page_table_stride + j] when page_table != NULL and
+ * phys = j otherwise. Contiguous [B, Hkv, nb]: seq_stride = Hkv*nb,
+ * block_stride = 1, head_stride = nb. Paged [P, Hkv]: seq_stride = 0,
+ * block_stride = Hkv, head_stride = 1, num_pages = P. `extent` = records
+ * addressable from `records`. `records` must be 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+#define BSA_QIDX_RECORD_BYTES 576
+
+typedef enum { BSA_IDX_FP4 = 1, BSA_IDX_INT4 = 2 } bsa_idx_format_t;
+
+typedef struct {
+  void* records;             /* device, 576-byte records as above */
+  float* gscale;             /* device, one float: the cache scale g */
+  int64_t seq_stride;
+  int64_t block_stride;
+  int64_t head_stride;
+  const int32_t* page_table; /* [B, page_table_stride] or NULL */
+  int32_t page_table_stride;
+  int32_t num_pages;         /* used when page_table != NULL */
+  int64_t extent;            /* records */
+  int32_t format;            /* bsa_idx_format_t */
+} bsa_qcache_t;
+
+/* Quantise the bf16 index keys k_idx (width r = 16) of every token t < seq_lens[b]
+ * (decode problems) into `out`, writing every record of blocks [0, ceil(T_b/64))
+ * and *out.gscale. qmax = 6 (FP4) or 7 (INT4). Every step is float32 with
+ * round-to-nearest-even:
+ *   1. A = max |k| over all those tokens; g = A / (qmax * 448), or 1 when A = 0;
+ *   2. per token: a = max_c |k[c]|, s = (a / qmax) / g; scale = the E4M3 value
+ *      nearest to s (ties to the even mantissa), 448 when s >= 448;
+ *   3. S = e4m3(scale); if S = 0 every magnitude is 0; else t = S * g and per
+ *      element m_c = the magnitude nearest to |k[c] / t| (ties to the even index),
+ *      at most 7; the sign bit is the sign bit of k[c].
+ * Runs three kernels on `stream` and uses *out.gscale as scratch in between. */
+bsa_status_t bsa_quantize_index_keys(const bsa_problem_t* prob, bsa_cache_t k_idx,
+                                     bsa_qcache_t out, int32_t* dev_status, void* stream);
+
+/* Step 1 (decode) on a 4-bit index-key cache: as bsa_score_blocks, with the index
+ * keys of `k_idx` dequantised exactly (codes and scales are exact in bf16; the
+ * E4M3 scale and g multiply the head sum, ReLU being positively homogeneous).
+ * Prefill problems return BSA_ERR_UNSUPPORTED. */
+bsa_status_t bsa_score_blocks_q(const bsa_problem_t* prob, const void* q_idx, bsa_qcache_t k_idx,
+                                float* block_scores, int32_t* dev_status, void* stream);
+
 /* Size of the fixed device scratch array used by bsa_decode_noalloc (8 MiB). */
 #define BSA_NOALLOC_SCRATCH_BYTES (8u << 20)
 

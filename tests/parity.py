@@ -87,8 +87,9 @@ def attention_errors(o_f32_dev, o_bf16_dev, lse_dev, o_ref, lse_ref):
     rel_l2 = float(np.linalg.norm(o32 - ref) / max(np.linalg.norm(ref), 1e-300)) if o32.size else 0.0
     lse_d = np.asarray(lse_dev, dtype=np.float64)
     lse_r = np.asarray(lse_ref, dtype=np.float64)
-    both_inf = np.isinf(lse_d) & np.isinf(lse_r)
-    lse_err = float(np.max(np.where(both_inf, 0.0, np.abs(lse_d - lse_r)))) if lse_d.size else 0.0
+    both_inf = np.isinf(lse_d) & np.isinf(lse_r) & (np.sign(lse_d) == np.sign(lse_r))
+    diff = np.abs(np.where(both_inf, 0.0, lse_d) - np.where(both_inf, 0.0, lse_r))
+    lse_err = float(np.max(diff)) if lse_d.size else 0.0
     return {"max_abs": max_abs, "rel_l2": rel_l2, "lse_abs": lse_err}
 
 

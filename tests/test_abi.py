@@ -93,3 +93,30 @@ def test_null_pointers_rejected_before_launch(lib):
 def test_status_strings(lib):
     for s in range(5):
         assert bsa.bsa_status_string(s)
+
+
+def _qcache(fmt=bsa.IDX_FP4, records=0x10000, gscale=0x20000):
+    return bsa.CQCache(records, gscale, 2 * 64, 1, 64, None, 0, 0, 2 * 2 * 64, fmt)
+
+
+def _kcache(base=0x30000):
+    return bsa.CCache(base, 2 * 4096 * 16, 64 * 16, 4096 * 16, None, 0, 0, 2 * 2 * 4096 * 16)
+
+
+def test_qcache_entry_points_reject_on_host(lib):
+    """Host checks of the 4-bit index-key entry points (no pointer is dereferenced)."""
+    p = _prob().c()
+    pf = _prob(phase=bsa.PHASE_PREFILL).c()
+    # prefill problems are not supported by the 4-bit path
+    assert lib.bsa_score_blocks_q(ctypes.byref(pf), 0x40000, _qcache(), 0x50000, None,
+                                  None) == bsa.BSA_ERR_UNSUPPORTED
+    assert lib.bsa_quantize_index_keys(ctypes.byref(pf), _kcache(), _qcache(), None,
+                                       None) == bsa.BSA_ERR_UNSUPPORTED
+    # unknown format, missing scale, unaligned records
+    for bad in (_qcache(fmt=3), _qcache(gscale=None), _qcache(records=0x10008)):
+        assert lib.bsa_score_blocks_q(ctypes.byref(p), 0x40000, bad, 0x50000, None,
+                                      None) == bsa.BSA_ERR_INVALID_ARG
+        assert lib.bsa_quantize_index_keys(ctypes.byref(p), _kcache(), bad, None,
+                                           None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_score_blocks_q(ctypes.byref(p), None, _qcache(), 0x50000, None,
+                                  None) == bsa.BSA_ERR_INVALID_ARG
