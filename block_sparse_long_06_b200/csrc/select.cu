@@ -14,10 +14,12 @@
 //     integer counts only, so deterministic) of the key of the Kcap-th candidate,
 //     Kcap = the largest dynamic count the caps allow; equal keys are taken in
 //     ascending id order via a block-wide scan;
-//  3. when 0 < p < 1: the Kcap winners are sorted by (key, id) with a bitonic
+//  3. when 0 < p < 1: Z = sum of exp(S - M) over all candidates and W = the same
+//     sum over the Kcap winners (fp64, fixed reduction trees). If W < p * Z no
+//     prefix of the winners reaches p and all Kcap are kept (the common case when
+//     K_max binds). Otherwise the winners are sorted by (key, id) with a bitonic
 //     sort, their masses exp(S - M) are prefix-summed in fp64 along that order
-//     (fixed order, deterministic) and the first prefix reaching p * Z is cut,
-//     Z = sum of exp(S - M) over all candidates (fp64, fixed reduction tree);
+//     (fixed order, deterministic) and the first prefix reaching p * Z is cut;
 //  4. kept list = [0, c0) ++ ascending dynamic ids ++ [c1, end), -1 padded.
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
@@ -221,14 +223,19 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_
   // ---- 3. top-p cut inside the kcap winners ------------------------------------
   if (need_mass) {
     // total mass over the candidates (fp64, fixed order)
-    double z = 0.0;
+    double z = 0.0, wsum = 0.0;
     const double Md = static_cast<double>(M);
     const bool all_inf = !(M > -INFINITY);
     for (int t = seg0; t < seg1; ++t) {
       const float s = S[c0 + t];
-      z += all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
+      const double m = all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
+      z += m;
+      if ((flags[t >> 5] >> (t & 31)) & 1u) wsum += m;
     }
     double Z = block_allreduce<NT>(z, dscr, [](double x, double y) { return x + y; });
+    const double W = block_allreduce<NT>(wsum, dscr, [](double x, double y) { return x + y; });
+    // the winners' whole mass stays below p: every winner is kept, no order is needed
+    if (W < static_cast<double>(ph) * Z) goto emit;
     // compact winners in id order, then sort by (key, id)
     int nsel = 0;
     for (int t = seg0; t < seg1; ++t) nsel += (flags[t >> 5] >> (t & 31)) & 1u;
@@ -290,6 +297,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_
     __syncthreads();
   }
 
+emit:
   // ---- 4. kept list ----------------------------------------------------------
   int nsel = 0;
   for (int t = seg0; t < seg1; ++t) nsel += (flags[t >> 5] >> (t & 31)) & 1u;
