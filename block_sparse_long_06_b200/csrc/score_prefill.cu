@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(kWarps * 32) score_prefill_kernel(const ScoreP
   // query fragments: tq group tg (8 tokens), head pair hp
   uint32_t aq[2][HP][4];
   float w[HP][2];
-  float2 w0p[HP], w1p[HP];   // half the weights of the pair's two heads, duplicated for FFMA2
+  float2 w0p[HP], w1p[HP];   // first head's weight, half the second head's, duplicated for FFMA2
   const char* qbase = static_cast<const char*>(a.q_idx);
   const float dflt = 1.0f / static_cast<float>(a.G);
 #pragma unroll
@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(kWarps * 32) score_prefill_kernel(const ScoreP
   }
 #pragma unroll
   for (int hp = 0; hp < HP; ++hp) {
-    w0p[hp] = make_float2(0.5f * w[hp][0], 0.5f * w[hp][0]);
+    w0p[hp] = make_float2(w[hp][0], w[hp][0]);
     w1p[hp] = make_float2(0.5f * w[hp][1], 0.5f * w[hp][1]);
   }
   // query tokens of this lane that exist (a ragged last query block)
@@ -103,14 +103,16 @@ __global__ void __launch_bounds__(kWarps * 32) score_prefill_kernel(const ScoreP
 #pragma unroll
           for (int tg = 0; tg < 2; ++tg) {
             // u = (key 2*tig, key 2*tig + 1): two-wide FMAs, head by head in order.
-            // ReLU on the FMA pipe: c + |c| is exactly 2c for c > 0 and +0 otherwise, so
-            // (w/2) * (c + |c|) + u rounds exactly as w * ReLU(c) + u does.
+            // The ReLU of the pair's first head runs on the ALU pipe (max with 0), the
+            // second head's on the FMA pipe: c + |c| is exactly 2c for c > 0 and +0
+            // otherwise, so (w/2) * (c + |c|) + u rounds exactly as w * ReLU(c) + u.
+            // Splitting the two keeps both pipes busy.
             float2 u = make_float2(0.f, 0.f);
 #pragma unroll
             for (int hp = 0; hp < HP; ++hp) {
               float c[4] = {0.f, 0.f, 0.f, 0.f};
               mma_bf16(c, aq[tg][hp], kv.x, kv.y);
-              u = __ffma2_rn(w0p[hp], make_float2(c[0] + fabsf(c[0]), c[1] + fabsf(c[1])), u);
+              u = __ffma2_rn(w0p[hp], make_float2(fmaxf(c[0], 0.f), fmaxf(c[1], 0.f)), u);
               u = __ffma2_rn(w1p[hp], make_float2(c[2] + fabsf(c[2]), c[3] + fabsf(c[3])), u);
             }
             const bool qv = tg == 0 ? q0v : q1v;
