@@ -60,7 +60,7 @@ class CProblem(ctypes.Structure):
                 ("n_sink", ctypes.c_int32), ("n_local", ctypes.c_int32),
                 ("k_max", ctypes.c_int32), ("k_min", ctypes.c_int32), ("p", ctypes.c_float),
                 ("idx_scale", ctypes.c_float), ("attn_scale", ctypes.c_float),
-                ("head_w", ctypes.c_void_p)]
+                ("head_w", ctypes.c_void_p), ("head_p", ctypes.c_void_p)]
 
 
 _lib = None
@@ -141,6 +141,7 @@ class Problem:
     attn_scale: float = 0.0       # 0 -> 1/sqrt(d)
     seq_lens: Optional[torch.Tensor] = None   # device int32 [B] (decode)
     head_w: Optional[torch.Tensor] = None     # device float32 [Hq]
+    head_p: Optional[torch.Tensor] = None     # device float32 [Hkv]: per-kv-head p (<= 0: local head)
 
     @property
     def G(self):
@@ -154,7 +155,7 @@ class Problem:
         return CProblem(self.phase, self.B, self.Hq, self.Hkv, self.d, self.r, self.block, self.T,
                         _ptr(self.seq_lens), self.n_sink, self.n_local, self.k_max, self.k_min,
                         float(self.p), float(self.idx_scale), float(self.attn_scale),
-                        _ptr(self.head_w))
+                        _ptr(self.head_w), _ptr(self.head_p))
 
 
 @dataclass

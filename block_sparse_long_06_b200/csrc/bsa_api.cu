@@ -231,6 +231,8 @@ bsa_status_t bsa_score_blocks(const bsa_problem_t* p, const void* q_idx, bsa_cac
     a.kidx = view(k_idx);
     a.seq_lens = p->seq_lens;
     a.head_w = p->head_w;
+    a.head_p = p->head_p;
+    a.k_min = p->k_min;
     a.scores = block_scores;
     a.status = dev_status;
     a.B = p->B;
@@ -249,6 +251,8 @@ bsa_status_t bsa_score_blocks(const bsa_problem_t* p, const void* q_idx, bsa_cac
     a.q_idx = q_idx;
     a.kidx = view(k_idx);
     a.head_w = p->head_w;
+    a.head_p = p->head_p;
+    a.k_min = p->k_min;
     a.scores = block_scores;
     a.status = dev_status;
     a.B = p->B;
@@ -297,6 +301,8 @@ bsa_status_t bsa_score_blocks_q(const bsa_problem_t* p, const void* q_idx, bsa_q
   a.kidx = qview(k_idx);
   a.seq_lens = p->seq_lens;
   a.head_w = p->head_w;
+    a.head_p = p->head_p;
+    a.k_min = p->k_min;
   a.scores = block_scores;
   a.status = dev_status;
   a.B = p->B;
@@ -339,6 +345,7 @@ bsa_status_t bsa_select_top_p(const bsa_problem_t* p, const float* block_scores,
   a.k_max = p->k_max;
   a.k_min = p->k_min;
   a.p = p->p;
+  a.head_p = p->head_p;
   cudaError_t e = bsa::launch_select(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e);
 }

@@ -23,6 +23,8 @@ struct ScoreDecodeArgs {
   CacheView kidx;             // width 16
   const int32_t* seq_lens;    // [B] or null
   const float* head_w;        // [Hq] or null
+  const float* head_p;        // [Hkv] or null; heads with p <= 0 (k_min = 0) are skipped
+  int k_min;
   float* scores;              // [B*Hkv, nb_max]
   int32_t* status;
   int B, Hq, Hkv, G, T, nb_max, chunks_per_row;
@@ -48,6 +50,8 @@ struct ScorePrefillArgs {
   const void* q_idx;          // [B, Hq, T, 16] bf16
   CacheView kidx;             // width 16
   const float* head_w;
+  const float* head_p;        // [Hkv] or null; heads with p <= 0 (k_min = 0) are skipped
+  int k_min;
   float* scores;              // [B*Hkv, nqb, nqb]
   int32_t* status;
   int B, Hq, Hkv, G, T, nqb;
@@ -63,6 +67,7 @@ struct SelectArgs {
   int phase, B, Hkv, T, nb_max, nqb, max_kept;
   int n_sink, n_local, k_max, k_min;
   float p;
+  const float* head_p;        // [Hkv] or null: per-head p
 };
 
 struct DecodeArgs {

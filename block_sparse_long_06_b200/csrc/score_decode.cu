@@ -41,9 +41,14 @@ constexpr int kThreads = (kConsumers + 1) * 32;
 struct StageInfo {
   int row;        // b * Hkv + g
   int j0;         // first block of the chunk
-  int Tb;         // tokens of sequence b
+  int Tb;         // tokens of sequence b; -1: a local head, nothing to score
   uint32_t ok;    // bit q: block j0 + q was copied
 };
+
+// A local head (p <= 0 with no K_min floor) keeps its reserved blocks only: no scores.
+BSA_DEVFN bool local_head(const ScoreDecodeArgs& a, int g) {
+  return a.head_p != nullptr && a.k_min == 0 && !(a.head_p[g] > 0.f);
+}
 
 // KF: key format, 0 = bf16 rows (32 B per token), 1 = FP4 / 2 = INT4 records.
 template <int KF>
@@ -155,57 +160,62 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
           break;
         }
         const int nb_row = (Tb + kBlock - 1) / kBlock;
-        const int nblk = max(0, min(kChunk, nb_row - j0));      // blocks of the chunk that exist
-        unsigned char* dst = ring + s * kStageBytes;
-        uint32_t ok = 0, bytes = 0;
-        if (KF != 0 && contiguous && nblk > 0) {
-          // adjacent whole records: one range check, one copy
-          int64_t rec;
-          if (block_record(a.kidx, b, g, j0, rec) && rec + nblk <= a.kidx.extent) {
-            ok = (1u << nblk) - 1u;
-            bytes = nblk * kBlockBytes;
-          }
-          info[s] = StageInfo{row, j0, Tb, ok};
-          mbar_arrive_expect_tx(&full[s], bytes);
-          if (ok) bulk_g2s(dst, kbase + rec * kBlockBytes, bytes, &full[s]);
-        } else if (KF != 0) {
-          int64_t recs[kChunk];
-          for (int q = 0; q < nblk; ++q)
-            if (block_record(a.kidx, b, g, j0 + q, recs[q])) {
-              ok |= 1u << q;
-              bytes += kBlockBytes;
-            }
-          info[s] = StageInfo{row, j0, Tb, ok};
-          mbar_arrive_expect_tx(&full[s], bytes);
-          for (int q = 0; q < nblk; ++q)
-            if (ok & (1u << q))
-              bulk_g2s(dst + q * kBlockBytes, kbase + recs[q] * kBlockBytes, kBlockBytes, &full[s]);
-        } else if (contiguous && nblk > 0) {
-          // the chunk's blocks are adjacent: one range check, one copy
-          const int rows = min(nblk * kBlock, Tb - j0 * kBlock);
-          int64_t off;
-          if (block_offset(a.kidx, b, g, j0, rows, off)) {
-            ok = (1u << nblk) - 1u;
-            bytes = rows * kR * 2;
-          }
-          info[s] = StageInfo{row, j0, Tb, ok};
-          mbar_arrive_expect_tx(&full[s], bytes);
-          if (ok) bulk_g2s(dst, kbase + off * 2, bytes, &full[s]);
+        if (local_head(a, g)) {
+          info[s] = StageInfo{row, j0, -1, 0u};
+          mbar_arrive(&full[s]);
         } else {
-          int64_t offs[kChunk];
-          int rows_q[kChunk];
-          for (int q = 0; q < nblk; ++q) {
-            rows_q[q] = min(kBlock, Tb - (j0 + q) * kBlock);
-            if (block_offset(a.kidx, b, g, j0 + q, rows_q[q], offs[q])) {
-              ok |= 1u << q;
-              bytes += rows_q[q] * kR * 2;
+          const int nblk = max(0, min(kChunk, nb_row - j0));      // blocks of the chunk that exist
+          unsigned char* dst = ring + s * kStageBytes;
+          uint32_t ok = 0, bytes = 0;
+          if (KF != 0 && contiguous && nblk > 0) {
+            // adjacent whole records: one range check, one copy
+            int64_t rec;
+            if (block_record(a.kidx, b, g, j0, rec) && rec + nblk <= a.kidx.extent) {
+              ok = (1u << nblk) - 1u;
+              bytes = nblk * kBlockBytes;
             }
+            info[s] = StageInfo{row, j0, Tb, ok};
+            mbar_arrive_expect_tx(&full[s], bytes);
+            if (ok) bulk_g2s(dst, kbase + rec * kBlockBytes, bytes, &full[s]);
+          } else if (KF != 0) {
+            int64_t recs[kChunk];
+            for (int q = 0; q < nblk; ++q)
+              if (block_record(a.kidx, b, g, j0 + q, recs[q])) {
+                ok |= 1u << q;
+                bytes += kBlockBytes;
+              }
+            info[s] = StageInfo{row, j0, Tb, ok};
+            mbar_arrive_expect_tx(&full[s], bytes);
+            for (int q = 0; q < nblk; ++q)
+              if (ok & (1u << q))
+                bulk_g2s(dst + q * kBlockBytes, kbase + recs[q] * kBlockBytes, kBlockBytes, &full[s]);
+          } else if (contiguous && nblk > 0) {
+            // the chunk's blocks are adjacent: one range check, one copy
+            const int rows = min(nblk * kBlock, Tb - j0 * kBlock);
+            int64_t off;
+            if (block_offset(a.kidx, b, g, j0, rows, off)) {
+              ok = (1u << nblk) - 1u;
+              bytes = rows * kR * 2;
+            }
+            info[s] = StageInfo{row, j0, Tb, ok};
+            mbar_arrive_expect_tx(&full[s], bytes);
+            if (ok) bulk_g2s(dst, kbase + off * 2, bytes, &full[s]);
+          } else {
+            int64_t offs[kChunk];
+            int rows_q[kChunk];
+            for (int q = 0; q < nblk; ++q) {
+              rows_q[q] = min(kBlock, Tb - (j0 + q) * kBlock);
+              if (block_offset(a.kidx, b, g, j0 + q, rows_q[q], offs[q])) {
+                ok |= 1u << q;
+                bytes += rows_q[q] * kR * 2;
+              }
+            }
+            info[s] = StageInfo{row, j0, Tb, ok};
+            mbar_arrive_expect_tx(&full[s], bytes);
+            for (int q = 0; q < nblk; ++q)
+              if (ok & (1u << q))
+                bulk_g2s(dst + q * kBlockBytes, kbase + offs[q] * 2, rows_q[q] * kR * 2, &full[s]);
           }
-          info[s] = StageInfo{row, j0, Tb, ok};
-          mbar_arrive_expect_tx(&full[s], bytes);
-          for (int q = 0; q < nblk; ++q)
-            if (ok & (1u << q))
-              bulk_g2s(dst + q * kBlockBytes, kbase + offs[q] * 2, rows_q[q] * kR * 2, &full[s]);
         }
         // next item
         j0 += kChunk;
@@ -240,6 +250,11 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
     }
     const StageInfo in = info[s];
     const int j = in.j0 + warp;
+    if (in.Tb < 0) {   // local head: release the stage, write nothing
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      continue;
+    }
     if (in.row != cur_row) {
       cur_row = in.row;
       const int b = in.row / a.Hkv, g = in.row - b * a.Hkv;

@@ -40,6 +40,7 @@ __global__ void __launch_bounds__(kWarps * 32) score_prefill_kernel(const ScoreP
   const int bg = static_cast<int>(blockIdx.x) % BH;
   const int b = bg / a.Hkv, g = bg % a.Hkv;
   if (i <= 0) return;
+  if (a.head_p != nullptr && a.k_min == 0 && !(a.head_p[g] > 0.f)) return;   // local head
 
   // query fragments: tq group tg (8 tokens), head pair hp
   uint32_t aq[2][HP][4];

@@ -6,7 +6,9 @@
 //  (histogram thresholding instead of a sort); HGA, Central mechanism §2 for
 //  the prefill diagonal block.)
 //
-// One CTA per row: decode row = (b, g); prefill row = (b, g, query block i).
+// One CTA per row: decode row = (b, g); prefill row = (b, g, query block i). The
+// row's p is that of its kv head when per-head values are given (RTPurbo,
+// Methodology §1: local heads keep their reserved blocks only).
 // The candidates form one contiguous id range [c0, c1) in both phases. Steps:
 //  1. keys: 32-bit order keys (smaller key = higher score; -0 folded into +0,
 //     NaN last) staged in shared memory; M = max score over the candidates;
@@ -120,7 +122,9 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_
   kcount = a.kept_count + row;
   const int nC = c1 - c0;
 
-  const float ph = a.p;
+  // top-p of this row's kv head (local heads have p <= 0: reserved blocks only)
+  const int g_row = a.phase == BSA_PHASE_DECODE ? row % a.Hkv : (row / a.nqb) % a.Hkv;
+  const float ph = a.head_p ? a.head_p[g_row] : a.p;
   int kcap;  // largest number of dynamic blocks the caps allow
   const int kminC = min(a.k_min, nC);
   if (ph <= 0.f)

@@ -101,6 +101,12 @@ typedef struct {
   float idx_scale;          /* index score scale; 0 = 1/sqrt(r) */
   float attn_scale;         /* softmax scale; 0 = 1/sqrt(d) */
   const float* head_w;      /* device [Hq] non-negative index-head weights, or NULL = 1/G */
+  const float* head_p;      /* device [Hkv] top-p per kv head, or NULL = p for every head.
+                               A head with p <= 0 and k_min = 0 is a local head (RTPurbo,
+                               Methodology §1: local heads keep sinks + a sliding window,
+                               retrieval heads select dynamically): it keeps only its
+                               reserved blocks, and the scorers skip it (its block_scores
+                               are left unwritten). */
 } bsa_problem_t;
 
 /* Length of one kept list: decode n_sink + n_local + k_max; prefill
