@@ -186,6 +186,12 @@ BSA_DEVFN float2 unpack_bf16(uint32_t x) {
 }
 
 // Hardware base-2 exponential (MUFU), approximate, flush-to-zero.
+// Programmatic dependent launch: wait until the grids this one depends on have
+// completed and their writes are visible (a no-op for a normal launch). Kernels
+// launched with launch_pdl call it before touching any buffer an earlier kernel of
+// the stream reads or writes; the code before it only sets up shared memory.
+BSA_DEVFN void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Value of an E4M3 (FP8, bias 7, with subnormals) code; 0x7F (NaN) is never produced
 // by the index-key quantiser.
 BSA_DEVFN float e4m3_value(uint32_t code) {

@@ -100,6 +100,25 @@ struct PrefillArgs {
   float scale_log2;
 };
 
+// Launch with programmatic stream serialization: the kernel's CTAs may start while
+// the previous kernel of the stream drains; the kernel orders itself after it with
+// grid_dependency_wait(). Hides launch latency between the steps of the path.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Each launcher returns the cudaError_t of its launch.
 cudaError_t launch_score_decode(const ScoreDecodeArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_quantize_index(const QuantArgs& a, int num_sms, cudaStream_t s);

@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
+  grid_dependency_wait();   // kept lists come from the selection kernel
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------- producer
@@ -344,6 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // One warp per (b, h): combine the splits of its row.
 template <int D>
 __global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a) {
+  grid_dependency_wait();   // partials come from the attention kernel
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= a.B * a.Hq) return;
@@ -393,12 +395,12 @@ cudaError_t launch_dn(const DecodeArgs& a, const CUtensorMap& tk, const CUtensor
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = num_units < num_sms ? num_units : num_sms;
-  if (grid > 0) kern<<<grid, kThreads, smem, s>>>(a, tk, tv, num_units);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (grid > 0) {
+    e = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, a, tk, tv, num_units);
+    if (e != cudaSuccess) return e;
+  }
   const int warps = a.B * a.Hq;
-  lse_merge_kernel<D><<<(warps * 32 + 255) / 256, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(lse_merge_kernel<D>, dim3((warps * 32 + 255) / 256), dim3(256), 0, s, a);
 }
 
 }  // namespace

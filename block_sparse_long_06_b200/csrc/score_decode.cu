@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
     fence_mbar_init();
   }
   __syncthreads();
+  grid_dependency_wait();   // the previous step may still read the score buffer
 
   const int64_t per = (a.total_items + gridDim.x - 1) / gridDim.x;
   const int64_t it0 = static_cast<int64_t>(blockIdx.x) * per;
@@ -347,8 +348,7 @@ cudaError_t launch_fmt(const ScoreDecodeArgs& a, int num_sms, cudaStream_t s) {
   auto kern = (a.G > 8) ? score_decode_kernel<2, KF> : score_decode_kernel<1, KF>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>(ctas), kThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, s, a);
 }
 
 }  // namespace

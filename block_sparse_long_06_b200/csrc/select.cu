@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x;
+  grid_dependency_wait();   // scores come from the scoring kernel
 
   // ---- row geometry -------------------------------------------------------
   int nbr, c0, c1;
@@ -335,8 +336,7 @@ cudaError_t launch_nt(const SelectArgs& a, int rows, int max_nc, cudaStream_t s)
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  select_kernel<NT><<<rows, NT, smem, s>>>(a, max_nc, sort_n);
-  return cudaGetLastError();
+  return launch_pdl(select_kernel<NT>, dim3(rows), dim3(NT), smem, s, a, max_nc, sort_n);
 }
 
 }  // namespace
