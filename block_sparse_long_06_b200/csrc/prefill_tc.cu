@@ -425,15 +425,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tqa = U.i * kBlock + (ra & 63), tqb = U.i * kBlock + (rb & 63);
       float ma = -INFINITY, mb = -INFINITY;
       float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
-      // block id and mask mode of the current step (the next one is fetched a step ahead)
-      int blk = U.i, mode = 2;
-      if (U.cnt > 0) {
-        blk = klist[0];
-        mode = mode_of(a, U, blk);
-      }
+      // block ids and mask modes of 32 steps at a time, one step per lane (fetched and
+      // validated in parallel, off the per-step path), then read by shuffle
+      int blk_v = U.i, mode_v = 2;
       bool ok = true;
       for (int jj = 0; jj < n; ++jj, ++kc) {
-        const int blk_nx = jj + 1 < U.cnt ? klist[jj + 1] : U.i;
+        if ((jj & 31) == 0) {
+          const int js = jj + lane;
+          blk_v = js < U.cnt ? klist[js] : U.i;
+          mode_v = js < U.cnt ? mode_of(a, U, blk_v) : 2;
+        }
+        const int blk = __shfl_sync(0xffffffffu, blk_v, jj & 31);
+        const int mode = __shfl_sync(0xffffffffu, mode_v, jj & 31);
         const int buf = kc & 1;
         if (!warp_wait(&bars->s_full[t], kc & 1)) { ok = false; break; }
         tc::fence_after_sync();
@@ -542,8 +545,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->p_ready[t][buf]);
-        blk = blk_nx;
-        mode = jj + 1 < U.cnt ? mode_of(a, U, blk) : 2;
       }
       if (!ok || aborted(bars)) {
         if (lane == 0) set_abort(bars, a.status);
