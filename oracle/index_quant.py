@@ -129,6 +129,50 @@ def quantize_token(k: np.ndarray, g: np.float32, fmt: str) -> tuple[np.ndarray, 
     return codes | sign, sc
 
 
+def _nearest_even(grid: np.ndarray, x: np.ndarray, top: int) -> np.ndarray:
+    """Index of the grid value nearest to each x >= 0, ties to the even index,
+    clamped at `top` (x beyond the grid saturates)."""
+    i = np.clip(np.searchsorted(grid, x, side="left"), 1, len(grid) - 1)
+    lo, hi = grid[i - 1], grid[i]
+    dlo, dhi = x - lo, hi - x
+    pick = np.where(dlo < dhi, i - 1, np.where(dhi < dlo, i, np.where((i - 1) % 2 == 0, i - 1, i)))
+    pick = np.where(x <= grid[0], 0, pick)
+    return np.where(x >= grid[-1], top, pick)
+
+
+def quantize_rows(k: np.ndarray, g, fmt: str) -> tuple[np.ndarray, np.ndarray]:
+    """quantize_token over many tokens at once: k [N, 16] (bf16-exact values), the
+    same float32 steps elementwise. Returns codes [N, 16] and scale codes [N]."""
+    k = np.asarray(k, dtype=np.float32)
+    g = np.float32(g)
+    a = np.max(np.abs(k), axis=1).astype(np.float32)
+    s = ((a / np.float32(QMAX[fmt])).astype(np.float32) / g).astype(np.float32)
+    vals64 = _E4M3_VALS
+    sc_idx = _nearest_even(vals64, np.minimum(s.astype(np.float64), E4M3_MAX),
+                           len(vals64) - 1)
+    # ties to the even mantissa: the E4M3 table index parity is the mantissa parity
+    sc = _E4M3_CODES[sc_idx]
+    S = vals64[sc_idx].astype(np.float32)
+    sign = np.signbit(k).astype(np.int64) << 3
+    t = (S * g).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        x = np.abs((k / t[:, None]).astype(np.float32)).astype(np.float64)
+    mag = _nearest_even(MAGNITUDES[fmt], np.nan_to_num(x, nan=0.0, posinf=1e30), 7)
+    mag = np.where((S == 0)[:, None], 0, mag)
+    return mag.astype(np.int64) | sign, sc.astype(np.uint8)
+
+
+def cache_gscale(k_idx: np.ndarray, seq_lens, fmt: str) -> np.float32:
+    """Step 1 alone: g from the maximum |k| over the visible tokens."""
+    B, Hkv, T, _ = k_idx.shape
+    lens = [T] * B if seq_lens is None else [int(x) for x in seq_lens]
+    amax = np.float32(0.0)
+    for b in range(B):
+        if lens[b] > 0:
+            amax = max(amax, np.float32(np.max(np.abs(k_idx[b, :, :lens[b]]))))
+    return gscale_of(amax, fmt)
+
+
 def quantize_cache(k_idx: np.ndarray, seq_lens, fmt: str):
     """k_idx [B, Hkv, T, 16] (bf16-exact values), seq_lens [B] or None.
     Returns codes [B, Hkv, nb*64, 16] int, scale codes [B, Hkv, nb*64] uint8 and g;

@@ -145,3 +145,49 @@ def test_decode_on_quantised_cache_ragged_and_g8(fmt):
         step, xq = run_decode_q(w, x, fmt)
         rows = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
         parity.compare_decode_rows(w, xq, step, rows)
+
+
+class _RowKeys:
+    """Dequantised index keys of a few (b, g) rows of a full-size cache, indexable
+    like the k_idx tensor by the parity helpers."""
+
+    def __init__(self, rows):
+        self.rows = rows
+
+    def __getitem__(self, idx):
+        b, g, sl = idx
+        return self.rows[(b, g)][sl]
+
+
+@pytest.mark.parametrize("fmt", ["fp4"])
+def test_quantised_decode_full_size_sampled_rows(fmt):
+    """128K, B = 32 (the bench's decode workload) on the 4-bit cache: device bytes of
+    sampled rows equal the oracle's, and those rows match the oracle end to end."""
+    w = W.WORKLOADS["decode_b32_h32_t128k_paged"]
+    x = W.make_decode_inputs(w, "cuda")
+    prob, qc = quantize_on_device(w, x, fmt)
+    step = bsa.DecodeStep(prob)
+    _, K, V = bsa.caches_for(x)
+    step.run(x["q"], x["q_idx"], qc, K, V)
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    lens = x["seq_lens"].cpu().tolist()
+    g = iq.cache_gscale(x["k_idx"].float().cpu().numpy(), lens, fmt)
+    assert np.float32(qc.gscale.item()) == g
+    rows = [(0, 0), (5, 3), (31, 7)]
+    rec = qc.records.view(w.B, w.Hkv, w.nb, iq.RECORD_BYTES)
+    deq = {}
+    for (b, gg) in rows:
+        k = x["k_idx"][b, gg].float().cpu().numpy()
+        codes, scales = iq.quantize_rows(k, g, fmt)
+        nbp = w.nb * 64
+        c = np.zeros((nbp, 16), dtype=np.int64)
+        sc = np.zeros(nbp, dtype=np.uint8)
+        c[:lens[b]], sc[:lens[b]] = codes[:lens[b]], scales[:lens[b]]
+        ref = iq.pack_records(c[None, None], sc[None, None])[0, 0]
+        assert np.array_equal(rec[b, gg].cpu().numpy(), ref), (b, gg)
+        deq[(b, gg)] = torch.from_numpy(iq.dequantize(c, sc, g, fmt))
+    xq = {k_: v for k_, v in x.items() if k_ != "k_idx"}
+    xq["k_idx"] = _RowKeys(deq)
+    s = parity.compare_decode_rows(w, xq, step, rows)
+    print("4-bit full size", s)

@@ -165,3 +165,23 @@ def _e4m3_floor(s):
 def test_mutants_are_caught(name, over):
     assert _golden_check(iq)
     assert not _golden_check(_Mutant(**over)), name
+
+
+def test_vectorised_quantiser_agrees_with_token_form():
+    """quantize_rows (used on full-size caches) takes the same decisions as
+    quantize_token, which the goldens and torch pin."""
+    rng = np.random.default_rng(4)
+    k = _bf16(rng.standard_normal((2000, 16)) * rng.uniform(1e-5, 20.0, (2000, 1)))
+    k[0] = 0.0
+    k[1] = 2.0 ** -20
+    k[2, 5] = -0.0
+    G = json.load(open(GOLDEN))
+    for fmt in ("fp4", "int4"):
+        g = iq.gscale_of(np.max(np.abs(k)), fmt)
+        cv, sv = iq.quantize_rows(k, g, fmt)
+        for n in range(len(k)):
+            c, sc = iq.quantize_token(k[n], g, fmt)
+            assert sc == sv[n] and np.array_equal(c, cv[n]), (fmt, n)
+        gk = np.array(G[fmt]["k"], dtype=np.float32)
+        cg, sg = iq.quantize_rows(gk, np.float32(G[fmt]["g"]), fmt)
+        assert cg.tolist() == G[fmt]["codes"] and sg.tolist() == G[fmt]["scale_codes"]
