@@ -111,27 +111,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------- producer
+    // The warp resolves 32 kept entries at a time (block id, then the K and V rows
+    // through the page table), one per lane, so the dependent global loads overlap;
+    // lane 0 then issues the TMA copies of those blocks back to back.
     if (lane == 0) {
       prefetch_tensormap(&tmk);
       prefetch_tensormap(&tmv);
-      uint32_t it = 0;
-      bool ok_all = true;
-      for (int unit = blockIdx.x; unit < num_units && ok_all; unit += gridDim.x) {
-        const int row = unit / a.splits, sp = unit % a.splits;
-        const int b = row / a.Hkv, g = row % a.Hkv;
-        const int cnt = min(a.kept_count[row], a.max_kept);
-        const int e0 = sp * a.split_len, e1 = min(cnt, e0 + a.split_len);
-        const int Tb = seq_len(a, b);
-        const int nb = (Tb + kBlock - 1) / kBlock;
-        for (int e = e0; e < e1; ++e, ++it) {
-          const int s = it % S;
-          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
-            report(a.status, BSA_DEV_TIMEOUT);
-            ok_all = false;
-            break;
-          }
-          const int blk = a.kept[static_cast<int64_t>(row) * a.max_kept + e];
-          int64_t rk = -1, rv = -1;
+    }
+    uint32_t it = 0;
+    bool ok_all = true;
+    for (int unit = blockIdx.x; unit < num_units && ok_all; unit += gridDim.x) {
+      const int row = unit / a.splits, sp = unit % a.splits;
+      const int b = row / a.Hkv, g = row % a.Hkv;
+      const int cnt = min(a.kept_count[row], a.max_kept);
+      const int e0 = sp * a.split_len, e1 = min(cnt, e0 + a.split_len);
+      const int Tb = seq_len(a, b);
+      const int nb = (Tb + kBlock - 1) / kBlock;
+      for (int base = e0; base < e1 && ok_all; base += 32) {
+        const int e = base + lane;
+        int blk = -1;
+        int64_t rk = -1, rv = -1;
+        if (e < e1) {
+          blk = a.kept[static_cast<int64_t>(row) * a.max_kept + e];
           if (blk >= 0 && blk < nb) {
             const int rows = min(kBlock, Tb - blk * kBlock);
             rk = tile_row(a.k, b, g, blk, rows, D);
@@ -140,23 +141,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             report(a.status, BSA_DEV_BAD_KEPT);
           }
-          const bool ok = rk >= 0 && rv >= 0;
-          sinfo[s] = ok ? blk : -1;
-          unsigned char* st = ring + s * Cfg::kStageBytes;
-          if (ok) {
-            mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
+        }
+        const int n_here = min(32, e1 - base);
+        for (int q = 0; q < n_here; ++q, ++it) {
+          const int blk_q = __shfl_sync(0xffffffffu, blk, q);
+          const int64_t rk_q = __shfl_sync(0xffffffffu, rk, q);
+          const int64_t rv_q = __shfl_sync(0xffffffffu, rv, q);
+          if (lane == 0) {
+            const int s = it % S;
+            if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
+              report(a.status, BSA_DEV_TIMEOUT);
+              ok_all = false;
+            } else {
+              const bool ok = rk_q >= 0 && rv_q >= 0;
+              sinfo[s] = ok ? blk_q : -1;
+              unsigned char* st = ring + s * Cfg::kStageBytes;
+              if (ok) {
+                mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
 #pragma unroll
-            for (int x = 0; x < Cfg::kBoxes; ++x) {
-              tma_load_2d(st + x * 8192, &tmk, x * 64, static_cast<int32_t>(rk), &full[s]);
-              tma_load_2d(st + Cfg::kTileBytes + x * 8192, &tmv, x * 64, static_cast<int32_t>(rv),
-                          &full[s]);
+                for (int x = 0; x < Cfg::kBoxes; ++x) {
+                  tma_load_2d(st + x * 8192, &tmk, x * 64, static_cast<int32_t>(rk_q), &full[s]);
+                  tma_load_2d(st + Cfg::kTileBytes + x * 8192, &tmv, x * 64,
+                              static_cast<int32_t>(rv_q), &full[s]);
+                }
+              } else {
+                mbar_arrive(&full[s]);
+              }
             }
-          } else {
-            mbar_arrive(&full[s]);
           }
+          ok_all = __shfl_sync(0xffffffffu, ok_all ? 1 : 0, 0) != 0;
+          if (!ok_all) break;
         }
       }
-      // drain: wait until the consumers released every stage we filled (bounded)
+    }
+    // drain: wait until the consumers released every stage we filled (bounded)
+    if (lane == 0) {
       for (uint32_t k = 0; k < S && k < it; ++k) {
         const uint32_t j = it - 1 - k;
         mbar_wait(&empty[j % S], (j / S) & 1, 200000000ull);
