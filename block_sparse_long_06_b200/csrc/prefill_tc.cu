@@ -236,64 +236,100 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kWarpLoad) {
     // -------------------------------------------------------------- Q / K / V
+    // Lane 0 takes units and loads Q; the warp resolves 32 steps' key blocks at a time
+    // (one per lane: kept-list entry, validation, cache row), then lane 0 issues the
+    // K and V copies of those steps back to back.
     if (lane == 0) {
       prefetch_tensormap(&tmq);
       prefetch_tensormap(&tmk);
       prefetch_tensormap(&tmv);
-      uint32_t un = 0, kc = 0;
-      bool ok = true;
-      while (ok) {
-        int u = atomicAdd(unit_counter, 1);
+    }
+    uint32_t un = 0, kc = 0;
+    bool ok = true;
+    while (ok) {
+      const int slot = un & 1;
+      int u = -1;
+      if (lane == 0) {
+        u = atomicAdd(unit_counter, 1);
         if (u >= num_units) u = -1;
-        const int slot = un & 1;
-        if (!mbar_wait_sleep(&bars->info_empty[slot], ((un >> 1) & 1) ^ 1)) { ok = false; break; }
-        UnitInfo U = {u, 0, 0, 0, 0, 0};
-        if (u >= 0) U = unit_of(a, u);
-        bars->info[slot] = U;
-        mbar_arrive(&bars->info_full[slot]);
-        if (u < 0 || aborted(bars)) break;
-        const int32_t* klist =
-            a.kept + (static_cast<int64_t>(U.b * a.Hkv + U.g) * a.nqb + U.i) * a.max_kept;
-        if (!mbar_wait_sleep(&bars->q_empty, (un & 1) ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&bars->q_full, ntiles * 2 * C::kHalves * 8192);
-        for (int t = 0; t < ntiles; ++t)
-          for (int hh = 0; hh < 2; ++hh) {
-            const int h = U.g * a.G + row_head(a, U.hq, t, hh * 64);
-            const int32_t qr = static_cast<int32_t>((static_cast<int64_t>(U.b) * a.Hq + h) * a.T +
-                                                    U.i * kBlock);
-            for (int x = 0; x < C::kHalves; ++x)
-              tma_load_2d(smem + t * C::kTile + x * C::kSlab + hh * 8192, &tmq, x * 64, qr,
-                          &bars->q_full);
-          }
-        const int n = U.cnt > 0 ? U.cnt : 1;
-        const int32_t vrow0 = static_cast<int32_t>((static_cast<int64_t>(U.b) * a.Hkv + U.g) * a.Tpad);
-        for (int jj = 0; jj < n; ++jj, ++kc) {
-          int blk = U.i;
-          int64_t rk = -1;
-          if (jj < U.cnt) {
-            blk = klist[jj];
-            rk = krow_of(a.k, a, U.b, U.g, blk, U.i);
-            if (rk < 0)
-              report(a.status, blk < 0 || blk > U.i ? BSA_DEV_BAD_KEPT : BSA_DEV_BAD_PAGE);
-          }
-          if (rk < 0) {
-            blk = U.i;   // load the always-valid diagonal block; its columns are masked
-            rk = krow_of(a.k, a, U.b, U.g, blk, U.i);
-            if (rk < 0) rk = 0;
-          }
-          const int s = kc % NS;
-          if (!mbar_wait_sleep(&bars->kv_empty[s], ((kc / NS) & 1) ^ 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars->kv_full[s], C::kStage);
-          unsigned char* st = smem + C::kOffKV + s * C::kStage;
-          for (int x = 0; x < C::kHalves; ++x)
-            tma_load_2d(st + x * 8192, &tmk, x * 64, static_cast<int32_t>(rk), &bars->kv_full[s]);
-          for (int x = 0; x < C::kHalves; ++x)
-            tma_load_2d(st + C::kBlk + x * 8192, &tmv, x * 64, vrow0 + blk * kBlock,
-                        &bars->kv_full[s]);
+        if (!mbar_wait_sleep(&bars->info_empty[slot], ((un >> 1) & 1) ^ 1)) {
+          ok = false;
+        } else {
+          UnitInfo U0 = {u, 0, 0, 0, 0, 0};
+          if (u >= 0) U0 = unit_of(a, u);
+          bars->info[slot] = U0;
+          mbar_arrive(&bars->info_full[slot]);
         }
-        if (!ok) break;
-        ++un;
       }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (!ok || u < 0 || aborted(bars)) break;
+      __syncwarp();
+      const UnitInfo U = bars->info[slot];
+      const int32_t* klist =
+          a.kept + (static_cast<int64_t>(U.b * a.Hkv + U.g) * a.nqb + U.i) * a.max_kept;
+      if (lane == 0) {
+        if (!mbar_wait_sleep(&bars->q_empty, (un & 1) ^ 1)) {
+          ok = false;
+        } else {
+          mbar_arrive_expect_tx(&bars->q_full, ntiles * 2 * C::kHalves * 8192);
+          for (int t = 0; t < ntiles; ++t)
+            for (int hh = 0; hh < 2; ++hh) {
+              const int h = U.g * a.G + row_head(a, U.hq, t, hh * 64);
+              const int32_t qr = static_cast<int32_t>(
+                  (static_cast<int64_t>(U.b) * a.Hq + h) * a.T + U.i * kBlock);
+              for (int x = 0; x < C::kHalves; ++x)
+                tma_load_2d(smem + t * C::kTile + x * C::kSlab + hh * 8192, &tmq, x * 64, qr,
+                            &bars->q_full);
+            }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      const int n = U.cnt > 0 ? U.cnt : 1;
+      const int32_t vrow0 = static_cast<int32_t>((static_cast<int64_t>(U.b) * a.Hkv + U.g) * a.Tpad);
+      for (int base = 0; base < n && ok; base += 32) {
+        const int jj = base + lane;
+        int blk = U.i;
+        int64_t rk = -1;
+        if (jj < U.cnt) {
+          blk = klist[jj];
+          rk = krow_of(a.k, a, U.b, U.g, blk, U.i);
+          if (rk < 0)
+            report(a.status, blk < 0 || blk > U.i ? BSA_DEV_BAD_KEPT : BSA_DEV_BAD_PAGE);
+        }
+        if (rk < 0) {
+          blk = U.i;   // load the always-valid diagonal block; its columns are masked
+          rk = krow_of(a.k, a, U.b, U.g, blk, U.i);
+          if (rk < 0) rk = 0;
+        }
+        const int n_here = min(32, n - base);
+        for (int q = 0; q < n_here; ++q, ++kc) {
+          const int blk_q = __shfl_sync(0xffffffffu, blk, q);
+          const int64_t rk_q = __shfl_sync(0xffffffffu, rk, q);
+          if (lane == 0) {
+            const int s = kc % NS;
+            if (!mbar_wait_sleep(&bars->kv_empty[s], ((kc / NS) & 1) ^ 1)) {
+              ok = false;
+            } else {
+              mbar_arrive_expect_tx(&bars->kv_full[s], C::kStage);
+              unsigned char* st = smem + C::kOffKV + s * C::kStage;
+              for (int x = 0; x < C::kHalves; ++x)
+                tma_load_2d(st + x * 8192, &tmk, x * 64, static_cast<int32_t>(rk_q),
+                            &bars->kv_full[s]);
+              for (int x = 0; x < C::kHalves; ++x)
+                tma_load_2d(st + C::kBlk + x * 8192, &tmv, x * 64, vrow0 + blk_q * kBlock,
+                            &bars->kv_full[s]);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+        }
+      }
+      if (!ok) break;
+      ++un;
+    }
+    if (lane == 0) {
       if (!ok) set_abort(bars, a.status);
       // copies in flight must land before the CTA exits (bounded)
       for (uint32_t k = (kc > NS ? kc - NS : 0); k < kc; ++k)
