@@ -220,6 +220,12 @@ def run_ours(args, world, rank, local):
     if do_pf:
         xp = W.make_prefill_inputs(wp, dev)
         pprob = bsa.problem_for(wp, head_w=xp["head_w"])
+        if args.idx_heads == 1:
+            # one index head per kv group: the bf16 mean of the group's index queries
+            qi = xp["q_idx"]
+            xp["q_idx"] = qi.float().reshape(wp.B, wp.Hkv, wp.G, *qi.shape[2:]).mean(2) \
+                .to(torch.bfloat16).contiguous()
+            pprob.idx_heads, pprob.head_w = 1, None
         pf = bsa.Prefill(pprob, device=dev, keep_f32=False)
         pk_idx = bsa.contiguous_cache(xp["k_idx"])
         pK = bsa.contiguous_cache(xp["K"])
@@ -341,6 +347,7 @@ def run_ours(args, world, rank, local):
         config["index_cache"] = args.index_cache
     if do_pf:
         config["prefill"] = describe(wp)
+        config["index_heads_per_group"] = 1 if args.idx_heads == 1 else wp.G
     config["l2"] = ("decode inputs exceed L2; a 256 MB buffer is written before each prefill")
     config["parallelism"] = f"dp{world} (independent sequences per GPU)"
     # kernels per step: decode = scorer, selection, split-K attention, LSE merge;
@@ -502,6 +509,9 @@ def main():
     ap.add_argument("--prefill-workload", default=PREFILL_WL, choices=sorted(
         k for k, v in W.WORKLOADS.items() if v.phase == "prefill"))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--idx-heads", type=int, choices=[0, 1], default=0,
+                    help="prefill index heads per kv group: 0 = one per query head (the "
+                         "method as configured), 1 = one per group (compact indexer)")
     ap.add_argument("--index-cache", choices=["bf16", "fp4", "int4"], default="bf16",
                     help="decode index-key cache: bf16 (the method as configured) or the "
                          "4-bit microscaled selector cache")

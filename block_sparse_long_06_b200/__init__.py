@@ -60,7 +60,8 @@ class CProblem(ctypes.Structure):
                 ("n_sink", ctypes.c_int32), ("n_local", ctypes.c_int32),
                 ("k_max", ctypes.c_int32), ("k_min", ctypes.c_int32), ("p", ctypes.c_float),
                 ("idx_scale", ctypes.c_float), ("attn_scale", ctypes.c_float),
-                ("head_w", ctypes.c_void_p), ("head_p", ctypes.c_void_p)]
+                ("head_w", ctypes.c_void_p), ("head_p", ctypes.c_void_p),
+                ("idx_heads", ctypes.c_int32)]
 
 
 _lib = None
@@ -142,6 +143,7 @@ class Problem:
     seq_lens: Optional[torch.Tensor] = None   # device int32 [B] (decode)
     head_w: Optional[torch.Tensor] = None     # device float32 [Hq]
     head_p: Optional[torch.Tensor] = None     # device float32 [Hkv]: per-kv-head p (<= 0: local head)
+    idx_heads: int = 0                        # 0: an index head per query head; 1: one per kv group
 
     @property
     def G(self):
@@ -155,7 +157,7 @@ class Problem:
         return CProblem(self.phase, self.B, self.Hq, self.Hkv, self.d, self.r, self.block, self.T,
                         _ptr(self.seq_lens), self.n_sink, self.n_local, self.k_max, self.k_min,
                         float(self.p), float(self.idx_scale), float(self.attn_scale),
-                        _ptr(self.head_w), _ptr(self.head_p))
+                        _ptr(self.head_w), _ptr(self.head_p), int(self.idx_heads))
 
 
 @dataclass

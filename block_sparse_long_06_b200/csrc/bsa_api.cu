@@ -92,8 +92,14 @@ bsa_status_t check_problem(const bsa_problem_t* p) {
   if (nblocks(p->T) > 32768) return BSA_ERR_UNSUPPORTED;
   if (p->phase == BSA_PHASE_PREFILL && p->seq_lens != nullptr) return BSA_ERR_UNSUPPORTED;
   if (p->phase == BSA_PHASE_PREFILL && p->T <= 0) return BSA_ERR_INVALID_ARG;
+  if (p->idx_heads != 0 && p->idx_heads != 1 && p->idx_heads != p->Hq / p->Hkv)
+    return BSA_ERR_UNSUPPORTED;
   return BSA_OK;
 }
+
+// Index heads per kv group: one per query head (the default) or one per group
+// (SparDA, Main innovations §2: a compact indexer with one head per GQA group).
+int idx_group(const bsa_problem_t* p) { return p->idx_heads == 1 ? 1 : p->Hq / p->Hkv; }
 
 float idx_scale_of(const bsa_problem_t* p) {
   return p->idx_scale > 0.f ? p->idx_scale : 1.0f / std::sqrt(static_cast<float>(p->r));
@@ -221,7 +227,6 @@ bsa_status_t bsa_score_blocks(const bsa_problem_t* p, const void* q_idx, bsa_cac
   if (st != BSA_OK) return st;
   if (q_idx == nullptr || block_scores == nullptr || !aligned16(q_idx)) return BSA_ERR_INVALID_ARG;
   if ((st = check_cache(k_idx, p, p->r, false)) != BSA_OK) return st;
-  const int G = p->Hq / p->Hkv;
   const int num_sms = num_sms_current();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
@@ -236,9 +241,9 @@ bsa_status_t bsa_score_blocks(const bsa_problem_t* p, const void* q_idx, bsa_cac
     a.scores = block_scores;
     a.status = dev_status;
     a.B = p->B;
-    a.Hq = p->Hq;
+    a.G = idx_group(p);
+    a.Hq = p->Hkv * a.G;   // index heads: q_idx rows and head weights
     a.Hkv = p->Hkv;
-    a.G = G;
     a.T = p->T;
     a.nb_max = nblocks(p->T);
     const int cb = bsa::score_decode_chunk_blocks();
@@ -256,9 +261,9 @@ bsa_status_t bsa_score_blocks(const bsa_problem_t* p, const void* q_idx, bsa_cac
     a.scores = block_scores;
     a.status = dev_status;
     a.B = p->B;
-    a.Hq = p->Hq;
+    a.G = idx_group(p);
+    a.Hq = p->Hkv * a.G;   // index heads: q_idx rows and head weights
     a.Hkv = p->Hkv;
-    a.G = G;
     a.T = p->T;
     a.nqb = nblocks(p->T);
     a.idx_scale = idx_scale_of(p);
@@ -306,9 +311,9 @@ bsa_status_t bsa_score_blocks_q(const bsa_problem_t* p, const void* q_idx, bsa_q
   a.scores = block_scores;
   a.status = dev_status;
   a.B = p->B;
-  a.Hq = p->Hq;
+  a.G = idx_group(p);
+  a.Hq = p->Hkv * a.G;   // index heads: q_idx rows and head weights
   a.Hkv = p->Hkv;
-  a.G = p->Hq / p->Hkv;
   a.T = p->T;
   a.nb_max = nblocks(p->T);
   const int cb = bsa::score_decode_chunk_blocks();

@@ -141,6 +141,92 @@ __global__ void __launch_bounds__(kWarps * 32) score_prefill_kernel(const ScoreP
   }
 }
 
+// One index head per group (G = 1: SparDA's compact indexer, or Hq = Hkv). With a
+// single weight w >= 0, max over pairs of w ReLU(q.k) = w ReLU(max over pairs of q.k)
+// exactly (rounding of w * x is monotone in x), so the per-pair epilogue is one max.
+// MMA rows are 16 query tokens (tokens gid and gid + 8 of the warp's 16).
+__global__ void __launch_bounds__(kWarps * 32) score_prefill_g1_kernel(const ScorePrefillArgs a) {
+  __shared__ float pm[kWarps][kBatch];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int BH = a.B * a.Hkv;
+  const int i = a.nqb - 1 - static_cast<int>(blockIdx.x) / BH;  // heavy rows first
+  const int bg = static_cast<int>(blockIdx.x) % BH;
+  const int b = bg / a.Hkv, g = bg % a.Hkv;
+  if (i <= 0) return;
+  if (a.head_p != nullptr && a.k_min == 0 && !(a.head_p[g] > 0.f)) return;   // local head
+  const float w = a.head_w ? a.head_w[g] : 1.0f;
+  const char* qbase = static_cast<const char*>(a.q_idx);
+  uint32_t aq[4] = {0u, 0u, 0u, 0u};
+  const int tq0 = i * kBlock + 16 * warp + gid, tq1 = tq0 + 8;
+  const bool q0v = tq0 < a.T, q1v = tq1 < a.T;
+  if (q0v) {
+    const uint2 x = *reinterpret_cast<const uint2*>(
+        qbase + (((static_cast<int64_t>(b) * a.Hq + g) * a.T + tq0) * kR + 4 * tig) * 2);
+    aq[0] = x.x;
+    aq[2] = x.y;
+  }
+  if (q1v) {
+    const uint2 x = *reinterpret_cast<const uint2*>(
+        qbase + (((static_cast<int64_t>(b) * a.Hq + g) * a.T + tq1) * kR + 4 * tig) * 2);
+    aq[1] = x.x;
+    aq[3] = x.y;
+  }
+  const char* kbase = static_cast<const char*>(a.kidx.base);
+  float* out = a.scores + (static_cast<int64_t>(bg) * a.nqb + i) * a.nqb;
+  for (int j0 = 0; j0 < i; j0 += kBatch) {
+    const int jn = min(kBatch, i - j0);
+    for (int jj = 0; jj < jn; ++jj) {
+      const int j = j0 + jj;
+      int64_t phys = j;
+      bool ok = true;
+      if (a.kidx.page_table != nullptr) {
+        phys = a.kidx.page_table[static_cast<int64_t>(b) * a.kidx.pt_stride + j];
+        ok = phys >= 0 && phys < a.kidx.num_pages;
+      }
+      const int64_t off = static_cast<int64_t>(b) * a.kidx.seq_stride + phys * a.kidx.block_stride +
+                          static_cast<int64_t>(g) * a.kidx.head_stride;
+      ok = ok && off >= 0 && off + kBlock * kR <= a.kidx.extent;
+      float m0 = -INFINITY, m1 = -INFINITY;
+      if (ok) {
+        const char* kb = kbase + off * 2;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          const uint2 kv = *reinterpret_cast<const uint2*>(kb + (nt * 8 + gid) * 32 + tig * 8);
+          float c[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_bf16(c, aq, kv.x, kv.y);
+          m0 = max3f(m0, c[0], c[1]);
+          m1 = max3f(m1, c[2], c[3]);
+        }
+        float mx = fmaxf(q0v ? m0 : -INFINITY, q1v ? m1 : -INFINITY);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) pm[warp][jj] = mx;
+      } else {
+        if (lane == 0) {
+          pm[warp][jj] = NAN;   // marks a failed block
+          if (warp == 0) report(a.status, BSA_DEV_BAD_PAGE);
+        }
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < jn) {
+      float m = pm[0][threadIdx.x];
+      bool bad = m != m;
+#pragma unroll
+      for (int ww = 1; ww < kWarps; ++ww) {
+        const float v = pm[ww][threadIdx.x];
+        bad = bad || v != v;
+        m = fmaxf(m, v);
+      }
+      const float sc = bad ? -INFINITY : a.idx_scale * (w * fmaxf(m, 0.f));
+      out[j0 + threadIdx.x] = sc;
+      if (!isfinite(sc)) report(a.status, BSA_DEV_NONFINITE);
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_score_prefill(const ScorePrefillArgs& a, int num_sms, cudaStream_t s) {
@@ -148,6 +234,10 @@ cudaError_t launch_score_prefill(const ScorePrefillArgs& a, int num_sms, cudaStr
   const int rows = a.B * a.Hkv * a.nqb;
   if (rows <= 0) return cudaSuccess;
   const int HP = (a.G + 1) / 2;
+  if (a.G == 1) {
+    score_prefill_g1_kernel<<<rows, kWarps * 32, 0, s>>>(a);
+    return cudaGetLastError();
+  }
   switch (HP) {
     case 1: score_prefill_kernel<1><<<rows, kWarps * 32, 0, s>>>(a); break;
     case 2: score_prefill_kernel<2><<<rows, kWarps * 32, 0, s>>>(a); break;

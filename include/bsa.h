@@ -107,6 +107,10 @@ typedef struct {
                                retrieval heads select dynamically): it keeps only its
                                reserved blocks, and the scorers skip it (its block_scores
                                are left unwritten). */
+  int32_t idx_heads;        /* index heads per kv group: 0 = one per query head (G; q_idx
+                               has Hq rows and head_w Hq entries), 1 = one per group (SparDA,
+                               Main innovations §2: a compact indexer; q_idx has Hkv rows,
+                               head_w Hkv entries or NULL = 1). Other values: unsupported. */
 } bsa_problem_t;
 
 /* Length of one kept list: decode n_sink + n_local + k_max; prefill
@@ -117,9 +121,11 @@ int32_t bsa_max_kept(const bsa_problem_t* prob);
 bsa_status_t bsa_workspace_size(const bsa_problem_t* prob, int32_t op, size_t* bytes);
 
 /* Step 1, block scores (SpotAttention, Methodology §1; RTPurbo, Methodology §2).
- * decode:  q_idx [B, Hq, r] bf16 -> block_scores [B, Hkv, nb] fp32, nb = ceil(T/64);
+ * decode:  q_idx [B, Hq, r] bf16 (Hkv rows when idx_heads = 1)
+ *          -> block_scores [B, Hkv, nb] fp32, nb = ceil(T/64);
  *          entries j >= ceil(seq_lens[b]/64) are set to -inf.
- * prefill: q_idx [B, Hq, T, r] bf16 -> block_scores [B, Hkv, nqb, nqb] fp32,
+ * prefill: q_idx [B, Hq, T, r] bf16 (Hkv rows when idx_heads = 1)
+ *          -> block_scores [B, Hkv, nqb, nqb] fp32,
  *          nqb = ceil(T/64); entry [i, j] written for j < i only.
  * k_idx addresses index keys (width r). */
 bsa_status_t bsa_score_blocks(const bsa_problem_t* prob, const void* q_idx, bsa_cache_t k_idx,

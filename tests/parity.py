@@ -113,15 +113,26 @@ def logical_rows(X: torch.Tensor, page_table, b: int, g: int, token_ids: np.ndar
     return X[pages, g, ids % 64]
 
 
+def index_heads(inputs, w, b, g, tail):
+    """Index queries and weights of group g: one index head per query head, or (with
+    inputs["idx_heads"] == 1) one per group, whose weight defaults to 1."""
+    if inputs.get("idx_heads", 0) == 1:
+        qi = f64(inputs["q_idx"][(b, slice(g, g + 1)) + tail])
+        hw = np.ones(1)
+        return 1, qi, hw
+    G = w.G
+    qi = f64(inputs["q_idx"][(b, slice(g * G, (g + 1) * G)) + tail])
+    return G, qi, f64(inputs["head_w"][g * G:(g + 1) * G])
+
+
 def oracle_decode_row(w, inputs, b, g, kept_override=None):
     """Oracle decode for row (b, g), gathering only the tokens it needs."""
     G = w.G
     lens = inputs["seq_lens"]
     T_b = int(lens[b])
     q_g = f64(inputs["q"][b, g * G:(g + 1) * G])
-    qi_g = f64(inputs["q_idx"][b, g * G:(g + 1) * G])
+    Gi, qi_g, hw = index_heads(inputs, w, b, g, (slice(None),))
     ki_g = f64(inputs["k_idx"][b, g, :T_b])
-    hw = f64(inputs["head_w"][g * G:(g + 1) * G])
     S = O.decode_block_scores(qi_g, ki_g, T_b, hw, 1.0 / math.sqrt(w.r))
     sel = O.select_decode(S, w.n_sink, w.n_local, w.p, w.k_max, w.k_min)
     kept = sel.kept if kept_override is None else list(kept_override)
@@ -177,11 +188,10 @@ def oracle_prefill_rows(w, inputs, b, g, rows, kept_override=None):
     G = w.G
     T = w.T
     q_g = f64(inputs["q"][b, g * G:(g + 1) * G, :T])
-    qi_g = f64(inputs["q_idx"][b, g * G:(g + 1) * G, :T])
+    _, qi_g, hw = index_heads(inputs, w, b, g, (slice(0, T),))
     ki_g = f64(inputs["k_idx"][b, g, :T])
     K_g = f64(inputs["K"][b, g, :T])
     V_g = f64(inputs["V"][b, g, :T])
-    hw = f64(inputs["head_w"][g * G:(g + 1) * G])
     return O.prefill_rows(q_g, qi_g, ki_g, K_g, V_g, T, hw, 1.0 / math.sqrt(w.r),
                           1.0 / math.sqrt(w.d), w.n_sink, w.n_local, w.p, w.k_max, w.k_min,
                           rows=rows, kept_override=kept_override)
