@@ -23,8 +23,18 @@
 //     sort, their masses exp(S - M) are prefix-summed in fp64 along that order
 //     (fixed order, deterministic) and the first prefix reaching p * Z is cut;
 //  4. kept list = [0, c0) ++ ascending dynamic ids ++ [c1, end), -1 padded.
+//
+// Long decode rows (more than 2048 candidates: few rows, each long, as at 1M
+// tokens) run on a cluster of up to 8 CTAs per row: each CTA holds a contiguous
+// slice of the candidates, and the cluster combines its maxima, radix histograms,
+// equal-key counts, masses and output offsets through distributed shared memory,
+// always in rank order, so every CTA takes the same decisions.
+#include <cooperative_groups.h>
+
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace bsa {
 namespace {
@@ -318,6 +328,283 @@ emit:
   if (tid == 0) *kcount = count;
 }
 
+template <int NT>
+__global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, int per_cta,
+                                                            int sort_n) {
+  constexpr int NW = NT / 32;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CL = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  extern __shared__ __align__(16) unsigned char smem[];
+  // layout: [sort buffer: sort_n u64][winners: sort_n u64][keys: skew(per_cta) u32]
+  //         [hist: copies*256 u32][flags: per_cta/32 u32]
+  uint64_t* sbuf = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* wbuf = sbuf + sort_n;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(wbuf + sort_n);
+  uint32_t* hist = keys + skew(per_cta) + 1;
+  uint32_t* flags = hist + kHistCopies * 256;
+  const int nflag_words = (per_cta + 31) / 32;
+  __shared__ double dscr[NW];
+  __shared__ uint32_t s_bucket_info[2];
+  __shared__ int s_hit;
+  __shared__ float s_fscr[NW];
+  __shared__ int s_iscr[NW];
+  // values each CTA publishes to the cluster
+  __shared__ float pub_max;
+  __shared__ uint32_t pub_hist[256];
+  __shared__ int pub_cnt, pub_k;
+  __shared__ double pub_z, pub_w;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = blockIdx.x / CL;
+  grid_dependency_wait();   // scores come from the scoring kernel
+
+  // ---- row geometry (decode rows) --------------------------------------------
+  const int b = row / a.Hkv;
+  int Tb = a.seq_lens ? a.seq_lens[b] : a.T;
+  Tb = Tb < 0 ? 0 : (Tb > a.T ? a.T : Tb);
+  const int nbr = (Tb + kBlock - 1) / kBlock;
+  const int c0 = min(a.n_sink, nbr);
+  const int c1 = max(c0, nbr - a.n_local);
+  const float* S = a.scores + static_cast<int64_t>(row) * a.nb_max;
+  int32_t* kept = a.kept + static_cast<int64_t>(row) * a.max_kept;
+  const int nC = c1 - c0;
+  const float ph = a.head_p ? a.head_p[row % a.Hkv] : a.p;
+  const int kminC = min(a.k_min, nC);
+  const int kcap = ph <= 0.f ? kminC : max(min(a.k_max, nC), kminC);
+  const bool need_mass = (ph > 0.f) && (ph < 1.f) && kcap > 0;
+  // this CTA's slice [lo, hi) of the candidates
+  const int lo = min(nC, rank * per_cta), hi = min(nC, lo + per_cta), n = hi - lo;
+
+  // ---- 1. keys and the cluster max ----------------------------------------------
+  float lmax = -INFINITY;
+  for (int t = tid; t < n; t += NT) {
+    const float s = S[c0 + lo + t];
+    keys[skew(t)] = order_key(s);
+    if (s == s) lmax = fmaxf(lmax, s);
+  }
+  for (int w = tid; w < nflag_words; w += NT) flags[w] = 0u;
+  lmax = block_allreduce<NT>(lmax, s_fscr, [](float x, float y) { return fmaxf(x, y); });
+  if (tid == 0) pub_max = lmax;
+  cluster.sync();
+  float M = -INFINITY;
+  for (int r = 0; r < CL; ++r) M = fmaxf(M, *cluster.map_shared_rank(&pub_max, r));
+
+  const int E = (n + NT - 1) / NT;
+  const int seg0 = min(n, tid * E), seg1 = min(n, seg0 + E);
+  int kdyn = 0;
+  if (kcap > 0 && kcap < nC) {
+    // ---- 2. radix select of the kcap-th key over the cluster's histograms ------
+    uint32_t prefix = 0u, pmask = 0u;
+    int rem = kcap;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int x = tid; x < kHistCopies * 256; x += NT) hist[x] = 0u;
+      __syncthreads();
+      uint32_t* h = hist + (warp % kHistCopies) * 256;
+      for (int t0 = 0; t0 < n; t0 += NT) {
+        const int t = t0 + tid;
+        uint32_t digit = 256u;
+        if (t < n) {
+          const uint32_t k = keys[skew(t)];
+          if ((k & pmask) == prefix) digit = (k >> shift) & 255u;
+        }
+        const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+        if (digit < 256u && lane == __ffs(peers) - 1) atomicAdd(&h[digit], __popc(peers));
+      }
+      __syncthreads();
+      for (int x = tid; x < 256; x += NT) {
+        uint32_t tot = 0;
+        for (int c = 0; c < kHistCopies; ++c) tot += hist[c * 256 + x];
+        pub_hist[x] = tot;
+      }
+      cluster.sync();
+      for (int x = tid; x < 256; x += NT) {
+        uint32_t tot = 0;
+        for (int r = 0; r < CL; ++r) tot += cluster.map_shared_rank(pub_hist, r)[x];
+        hist[x] = tot;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        uint32_t part = 0;
+        for (int q = 0; q < 8; ++q) part += hist[lane * 8 + q];
+        uint32_t inc = part;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t nn = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += nn;
+        }
+        const uint32_t exc = inc - part;
+        const bool here = (exc < static_cast<uint32_t>(rem)) && (inc >= static_cast<uint32_t>(rem));
+        if (here) {
+          uint32_t c = exc;
+          int bsel = lane * 8;
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t hq = hist[lane * 8 + q];
+            if (c + hq >= static_cast<uint32_t>(rem)) {
+              bsel = lane * 8 + q;
+              break;
+            }
+            c += hq;
+          }
+          s_bucket_info[0] = static_cast<uint32_t>(bsel);
+          s_bucket_info[1] = c;
+        }
+      }
+      __syncthreads();
+      prefix |= s_bucket_info[0] << shift;
+      pmask |= 255u << shift;
+      rem -= static_cast<int>(s_bucket_info[1]);
+      cluster.sync();   // every CTA has read pub_hist before the next pass writes it
+    }
+    // keys < prefix are in; among keys == prefix the `rem` lowest ids, counted
+    // across the cluster in rank (= id) order
+    int neq = 0;
+    for (int t = seg0; t < seg1; ++t) neq += (keys[skew(t)] == prefix);
+    int tot_eq;
+    int eq_base = block_exscan<NT>(neq, s_iscr, tot_eq);
+    if (tid == 0) pub_cnt = tot_eq;
+    cluster.sync();
+    for (int r = 0; r < rank; ++r) eq_base += *cluster.map_shared_rank(&pub_cnt, r);
+    for (int t = seg0; t < seg1; ++t) {
+      const uint32_t k = keys[skew(t)];
+      bool in = k < prefix;
+      if (k == prefix) in = (eq_base++ < rem);
+      if (in) atomicOr(&flags[t >> 5], 1u << (t & 31));
+    }
+    kdyn = kcap;
+    cluster.sync();   // pub_cnt may be written again
+  } else if (kcap > 0) {
+    for (int t = tid; t < n; t += NT) atomicOr(&flags[t >> 5], 1u << (t & 31));
+    kdyn = nC;
+  }
+  __syncthreads();
+
+  // ---- 3. top-p cut inside the kcap winners ------------------------------------
+  if (need_mass) {
+    double z = 0.0, wsum = 0.0;
+    const double Md = static_cast<double>(M);
+    const bool all_inf = !(M > -INFINITY);
+    for (int t = seg0; t < seg1; ++t) {
+      const float s = S[c0 + lo + t];
+      const double m = all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
+      z += m;
+      if ((flags[t >> 5] >> (t & 31)) & 1u) wsum += m;
+    }
+    const double zl = block_allreduce<NT>(z, dscr, [](double x, double y) { return x + y; });
+    const double wl = block_allreduce<NT>(wsum, dscr, [](double x, double y) { return x + y; });
+    if (tid == 0) {
+      pub_z = zl;
+      pub_w = wl;
+    }
+    cluster.sync();
+    double Z = 0.0, W = 0.0;
+    for (int r = 0; r < CL; ++r) {
+      Z += *cluster.map_shared_rank(&pub_z, r);
+      W += *cluster.map_shared_rank(&pub_w, r);
+    }
+    if (!(W < static_cast<double>(ph) * Z)) {
+      // the cut may fall inside the winners: rank 0 orders all of them
+      int nsel = 0;
+      for (int t = seg0; t < seg1; ++t) nsel += (flags[t >> 5] >> (t & 31)) & 1u;
+      int tot;
+      int pos = block_exscan<NT>(nsel, s_iscr, tot);
+      for (int t = seg0; t < seg1; ++t)
+        if ((flags[t >> 5] >> (t & 31)) & 1u)
+          wbuf[pos++] = (static_cast<uint64_t>(keys[skew(t)]) << 32) | static_cast<uint32_t>(lo + t);
+      if (tid == 0) pub_cnt = tot;
+      cluster.sync();
+      if (rank == 0) {
+        int off = 0;
+        for (int r = 0; r < CL; ++r) {
+          const int cr = *cluster.map_shared_rank(&pub_cnt, r);
+          const uint64_t* src = cluster.map_shared_rank(wbuf, r);
+          for (int x = tid; x < cr; x += NT) sbuf[off + x] = src[x];
+          off += cr;
+        }
+        for (int x = off + tid; x < sort_n; x += NT) sbuf[x] = ~0ull;
+        __syncthreads();
+        for (int kk = 2; kk <= sort_n; kk <<= 1) {
+          for (int j = kk >> 1; j > 0; j >>= 1) {
+            for (int x = tid; x < sort_n; x += NT) {
+              const int y = x ^ j;
+              if (y > x) {
+                const uint64_t u = sbuf[x], v = sbuf[y];
+                const bool asc = (x & kk) == 0;
+                if ((u > v) == asc) {
+                  sbuf[x] = v;
+                  sbuf[y] = u;
+                }
+              }
+            }
+            __syncthreads();
+          }
+        }
+        const int E2 = (kdyn + NT - 1) / NT;
+        const int q0 = min(kdyn, tid * E2), q1 = min(kdyn, q0 + E2);
+        double loc = 0.0;
+        for (int x = q0; x < q1; ++x) {
+          const float s = S[c0 + static_cast<int>(sbuf[x] & 0xffffffffu)];
+          loc += all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
+        }
+        double dtot;
+        double run = block_exscan<NT>(loc, dscr, dtot);
+        if (tid == 0) s_hit = 0x7fffffff;
+        __syncthreads();
+        const double target = static_cast<double>(ph) * Z;
+        for (int x = q0; x < q1; ++x) {
+          const float s = S[c0 + static_cast<int>(sbuf[x] & 0xffffffffu)];
+          run += all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
+          if (run >= target) {
+            atomicMin(&s_hit, x);
+            break;
+          }
+        }
+        __syncthreads();
+        const int capC = min(a.k_max, nC);
+        if (tid == 0) pub_k = (s_hit != 0x7fffffff) ? max(min(s_hit + 1, capC), kminC) : kdyn;
+      }
+      cluster.sync();
+      const int k = *cluster.map_shared_rank(&pub_k, 0);
+      for (int w = tid; w < nflag_words; w += NT) flags[w] = 0u;
+      __syncthreads();
+      const uint64_t* order = cluster.map_shared_rank(sbuf, 0);
+      for (int x = tid; x < k; x += NT) {
+        const int id = static_cast<int>(order[x] & 0xffffffffu);
+        if (id >= lo && id < hi) atomicOr(&flags[(id - lo) >> 5], 1u << ((id - lo) & 31));
+      }
+      kdyn = k;
+      cluster.sync();   // rank 0's order is no longer read; pub_cnt may be written again
+    }
+  }
+  __syncthreads();
+
+  // ---- 4. kept list: each CTA's ids after those of the lower ranks ----------------
+  int nsel = 0;
+  for (int t = seg0; t < seg1; ++t) nsel += (flags[t >> 5] >> (t & 31)) & 1u;
+  int tot;
+  int pos = block_exscan<NT>(nsel, s_iscr, tot);
+  if (tid == 0) pub_cnt = tot;
+  cluster.sync();
+  int below = 0, all = 0;
+  for (int r = 0; r < CL; ++r) {
+    const int v = *cluster.map_shared_rank(&pub_cnt, r);
+    if (r < rank) below += v;
+    all += v;
+  }
+  for (int t = seg0; t < seg1; ++t)
+    if ((flags[t >> 5] >> (t & 31)) & 1u) kept[c0 + below + pos++] = c0 + lo + t;
+  if (rank == 0) {
+    for (int x = tid; x < c0; x += NT) kept[x] = x;
+    const int nlocal = nbr - c1;
+    for (int x = tid; x < nlocal; x += NT) kept[c0 + all + x] = c1 + x;
+    const int count = c0 + all + nlocal;
+    for (int x = count + tid; x < a.max_kept; x += NT) kept[x] = -1;
+    if (tid == 0) a.kept_count[row] = count;
+  }
+  cluster.sync();   // no CTA leaves while another may still read its shared memory
+}
+
 int pow2_at_least(int x) {
   int p = 1;
   while (p < x) p <<= 1;
@@ -339,6 +626,39 @@ cudaError_t launch_nt(const SelectArgs& a, int rows, int max_nc, cudaStream_t s)
   return launch_pdl(select_kernel<NT>, dim3(rows), dim3(NT), smem, s, a, max_nc, sort_n);
 }
 
+// Long decode rows: a cluster of CL = 2..8 CTAs per row, each with <= 4096 candidates.
+template <int NT>
+cudaError_t launch_cluster(const SelectArgs& a, int rows, int max_nc, cudaStream_t s) {
+  int cl = 2;
+  while (cl < 8 && cl * 2048 < max_nc) cl *= 2;
+  const int per_cta = ((max_nc + cl - 1) / cl + 31) & ~31;
+  const int kcap_max = max(min(a.k_max, max_nc), min(a.k_min, max_nc));
+  const int sort_n = pow2_at_least(max(kcap_max, 2));
+  const int nflag_words = (per_cta + 31) / 32;
+  size_t smem = static_cast<size_t>(sort_n) * 16 + (static_cast<size_t>(skew(per_cta)) + 1) * 4 +
+                kHistCopies * 256 * 4 + (nflag_words + 1) * 4;
+  smem = (smem + 15) & ~static_cast<size_t>(15);
+  cudaError_t e = cudaFuncSetAttribute(select_cluster_kernel<NT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows * cl);
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, select_cluster_kernel<NT>, a, per_cta, sort_n);
+}
+
 }  // namespace
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
@@ -352,6 +672,11 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   }
   if (rows <= 0) return cudaSuccess;
   max_nc = max(max_nc, 1);
+  if (a.phase == BSA_PHASE_DECODE && max_nc > 2048) {
+    // few long rows: one cluster of CTAs per row
+    return max_nc <= 16384 ? launch_cluster<256>(a, rows, max_nc, s)
+                           : launch_cluster<512>(a, rows, max_nc, s);
+  }
   if (max_nc <= 2048) return launch_nt<256>(a, rows, max_nc, s);
   if (max_nc <= 8192) return launch_nt<512>(a, rows, max_nc, s);
   return launch_nt<1024>(a, rows, max_nc, s);

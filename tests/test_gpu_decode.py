@@ -148,3 +148,17 @@ def test_decode_full_size_sampled_rows(name):
     assert int(step.kept_count.max()) <= w.n_sink + w.n_local + w.k_max
     del x, step
     torch.cuda.empty_cache()
+
+
+# rows longer than 2048 candidates run the cluster selection (several CTAs per row)
+LONG = W.Workload("long_rows", "decode", B=3, Hq=8, Hkv=2, d=64, T=64 * 5000 + 17, paged=False,
+                  n_sink=2, n_local=3, p=0.9, k_max=300, hh_count=40, amp=3.0, seed=21,
+                  seq_lens=(64 * 5000 + 17, 64 * 3000 + 5, 90))
+
+
+@pytest.mark.parametrize("p,k_min", [(0.05, 0), (0.5, 4), (0.9, 0), (1.0, 0), (0.0, 7)])
+def test_decode_long_rows_cluster_select(p, k_min):
+    w = LONG.with_(p=p, k_min=k_min)
+    x = W.make_decode_inputs(w, "cpu")
+    step = run_decode(w, to_dev(x))
+    parity.compare_decode_rows(w, x, step, all_rows(w))
