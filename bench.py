@@ -55,9 +55,10 @@ def kernel_source_hash(files):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key, files):
+def ncu_traffic(kernel_key, files, workload):
     """Per-launch DRAM bytes from the committed ncu summary, if the kernel source
-    still matches the one the counters were taken on; else None."""
+    still matches the one the counters were taken on and the figure is for this
+    workload; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -65,6 +66,8 @@ def ncu_traffic(kernel_key, files):
         d = json.load(f)
     ent = d.get(kernel_key)
     if not ent or ent.get("source_hash") != kernel_source_hash(files):
+        return None
+    if ent.get("workload") != workload:
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -313,7 +316,7 @@ def run_ours(args, world, rank, local):
         files = ["decode_attn.cu", "bsa_common.cuh", "bsa_internal.h"]
         roof_dec = {"bound": "hbm", "kernel": "bsa_decode (split-K attention + LSE merge)",
                     "achieved": attn_gbs, "peak": hbm, "unit": "GB/s", "frac": attn_gbs / hbm,
-                    "traffic": ncu_traffic("decode_attn", files),
+                    "traffic": ncu_traffic("decode_attn", files, wd.name),
                     "peak_source": f"{peak_src} hbm_gbs (burst copy)",
                     "bytes_per_launch": by["attention"]}
     if do_pf:
@@ -327,7 +330,7 @@ def run_ours(args, world, rank, local):
         roof_pf = {"bound": "tensor", "kernel": "bsa_prefill (V->fp16 + attention)",
                    "achieved": pf_tflops / world, "peak": tflops_peak, "unit": "TFLOP/s",
                    "frac": pf_tflops / world / tflops_peak,
-                   "traffic": ncu_traffic("prefill_tc", files),
+                   "traffic": ncu_traffic("prefill_tc", files, wp.name),
                    "peak_source": f"{peak_src} bf16_tflops (burst)",
                    "flop_per_launch": flops}
 

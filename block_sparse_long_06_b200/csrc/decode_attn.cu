@@ -361,7 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// One warp per (b, h): combine the splits of its row.
+// One warp per (b, h): combine the splits of its row. The lanes read 32 splits'
+// (m, l) at once; the partial outputs of a chunk are then read with independent
+// loads (unrolled), added in split order.
 template <int D>
 __global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a) {
   grid_dependency_wait();   // partials come from the attention kernel
@@ -372,24 +374,35 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a) {
   const int g = h / a.G, hl = h % a.G;
   const int row = b * a.Hkv + g;
   constexpr int PER = D / 32;
+  const int64_t p0 = static_cast<int64_t>(row) * a.splits * a.G + hl;   // split s: p0 + s * G
   float M = -INFINITY;
-  for (int s = 0; s < a.splits; ++s) {
-    const int64_t pidx = static_cast<int64_t>(row * a.splits + s) * a.G + hl;
-    M = fmaxf(M, a.part_ml[pidx * 2]);
-  }
+  for (int s = lane; s < a.splits; s += 32) M = fmaxf(M, a.part_ml[(p0 + static_cast<int64_t>(s) * a.G) * 2]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   const float base = M == -INFINITY ? 0.f : M;
   float o[PER];
 #pragma unroll
   for (int q = 0; q < PER; ++q) o[q] = 0.f;
   float L = 0.f;
-  for (int s = 0; s < a.splits; ++s) {
-    const int64_t pidx = static_cast<int64_t>(row * a.splits + s) * a.G + hl;
-    const float f = ex2(a.part_ml[pidx * 2] - base);
-    L += a.part_ml[pidx * 2 + 1] * f;
-    const float* po = a.part_o + pidx * D;
+  for (int c = 0; c < a.splits; c += 32) {
+    const int s = c + lane;
+    float f = 0.f;
+    if (s < a.splits) {
+      const int64_t pidx = p0 + static_cast<int64_t>(s) * a.G;
+      f = ex2(a.part_ml[pidx * 2] - base);
+      L += a.part_ml[pidx * 2 + 1] * f;
+    }
+    const int nn = min(32, a.splits - c);
+#pragma unroll 4
+    for (int j = 0; j < nn; ++j) {
+      const float fj = __shfl_sync(0xffffffffu, f, j);
+      const float* po = a.part_o + (p0 + static_cast<int64_t>(c + j) * a.G) * D;
 #pragma unroll
-    for (int q = 0; q < PER; ++q) o[q] += po[lane + 32 * q] * f;
+      for (int q = 0; q < PER; ++q) o[q] += po[lane + 32 * q] * fj;
+    }
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
   const float inv = L > 0.f ? 1.0f / L : 0.f;
   const int64_t obase = (static_cast<int64_t>(b) * a.Hq + h) * D;
   __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o);

@@ -40,6 +40,7 @@ namespace bsa {
 namespace {
 
 constexpr int kHistCopies = 8;
+constexpr int kMaxCluster = 8;    // CTAs per long decode row, at most
 
 BSA_DEVFN uint32_t order_key(float s) {
   if (s != s) return 0xffffffffu;           // NaN: lowest priority
@@ -328,6 +329,15 @@ emit:
   if (tid == 0) *kcount = count;
 }
 
+// Writes `v` into slot `slot` of the array `box` of every CTA of the cluster. The
+// exchanges push rather than pull: remote stores do not stall the writer, and after
+// the next cluster barrier every CTA reads the values from its own shared memory
+// (a remote read costs about a thousand cycles).
+template <typename T>
+BSA_DEVFN void push_ranks(cg::cluster_group& cluster, T* box, int slot, int CL, T v) {
+  for (int r = 0; r < CL; ++r) *cluster.map_shared_rank(box + slot, r) = v;
+}
+
 template <int NT>
 __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, int per_cta,
                                                             int sort_n) {
@@ -350,13 +360,19 @@ __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, 
   __shared__ float s_fscr[NW];
   __shared__ int s_iscr[NW];
   // values each CTA publishes to the cluster
-  __shared__ float pub_max;
-  __shared__ uint32_t pub_hist[256];
+  // values the CTAs push to one another, slot = the writer's rank
+  __shared__ float rx_max[kMaxCluster];
+  __shared__ uint32_t rx_hist[2][kMaxCluster * 256];
+  __shared__ int rx_eq[kMaxCluster], rx_sel[kMaxCluster];
+  __shared__ double rx_z[kMaxCluster], rx_w[kMaxCluster];
+  // values read by pull (rare path)
   __shared__ int pub_cnt, pub_k;
-  __shared__ double pub_z, pub_w;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x / CL;
+  // every CTA of the cluster must be running before another writes into its shared
+  // memory: arrive now, wait just before the first push (the key loads run between)
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   grid_dependency_wait();   // scores come from the scoring kernel
 
   // ---- row geometry (decode rows) --------------------------------------------
@@ -376,7 +392,7 @@ __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, 
   // this CTA's slice [lo, hi) of the candidates
   const int lo = min(nC, rank * per_cta), hi = min(nC, lo + per_cta), n = hi - lo;
 
-  // ---- 1. keys and the cluster max ----------------------------------------------
+  // ---- 1. keys and the local max (published with the first exchange) -----------
   float lmax = -INFINITY;
   for (int t = tid; t < n; t += NT) {
     const float s = S[c0 + lo + t];
@@ -385,20 +401,25 @@ __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, 
   }
   for (int w = tid; w < nflag_words; w += NT) flags[w] = 0u;
   lmax = block_allreduce<NT>(lmax, s_fscr, [](float x, float y) { return fmaxf(x, y); });
-  if (tid == 0) pub_max = lmax;
-  cluster.sync();
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if (tid < CL) *cluster.map_shared_rank(&rx_max[rank], tid) = lmax;
   float M = -INFINITY;
-  for (int r = 0; r < CL; ++r) M = fmaxf(M, *cluster.map_shared_rank(&pub_max, r));
+  auto cluster_max = [&]() {
+    for (int r = 0; r < CL; ++r) M = fmaxf(M, rx_max[r]);
+  };
 
   const int E = (n + NT - 1) / NT;
   const int seg0 = min(n, tid * E), seg1 = min(n, seg0 + E);
   int kdyn = 0;
   if (kcap > 0 && kcap < nC) {
     // ---- 2. radix select of the kcap-th key over the cluster's histograms ------
+    // One cluster barrier per pass: the published histograms alternate between two
+    // buffers, so a pass never overwrites a copy that another CTA may still read.
     uint32_t prefix = 0u, pmask = 0u;
     int rem = kcap;
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 24 - 8 * pass;
+      uint32_t* rx = rx_hist[pass & 1];
       for (int x = tid; x < kHistCopies * 256; x += NT) hist[x] = 0u;
       __syncthreads();
       uint32_t* h = hist + (warp % kHistCopies) * 256;
@@ -416,12 +437,13 @@ __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, 
       for (int x = tid; x < 256; x += NT) {
         uint32_t tot = 0;
         for (int c = 0; c < kHistCopies; ++c) tot += hist[c * 256 + x];
-        pub_hist[x] = tot;
+        push_ranks(cluster, rx, rank * 256 + x, CL, tot);
       }
       cluster.sync();
+      if (pass == 0) cluster_max();
       for (int x = tid; x < 256; x += NT) {
         uint32_t tot = 0;
-        for (int r = 0; r < CL; ++r) tot += cluster.map_shared_rank(pub_hist, r)[x];
+        for (int r = 0; r < CL; ++r) tot += rx[r * 256 + x];
         hist[x] = tot;
       }
       __syncthreads();
@@ -455,7 +477,6 @@ __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, 
       prefix |= s_bucket_info[0] << shift;
       pmask |= 255u << shift;
       rem -= static_cast<int>(s_bucket_info[1]);
-      cluster.sync();   // every CTA has read pub_hist before the next pass writes it
     }
     // keys < prefix are in; among keys == prefix the `rem` lowest ids, counted
     // across the cluster in rank (= id) order
@@ -463,9 +484,9 @@ __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, 
     for (int t = seg0; t < seg1; ++t) neq += (keys[skew(t)] == prefix);
     int tot_eq;
     int eq_base = block_exscan<NT>(neq, s_iscr, tot_eq);
-    if (tid == 0) pub_cnt = tot_eq;
+    if (tid < CL) *cluster.map_shared_rank(&rx_eq[rank], tid) = tot_eq;
     cluster.sync();
-    for (int r = 0; r < rank; ++r) eq_base += *cluster.map_shared_rank(&pub_cnt, r);
+    for (int r = 0; r < rank; ++r) eq_base += rx_eq[r];
     for (int t = seg0; t < seg1; ++t) {
       const uint32_t k = keys[skew(t)];
       bool in = k < prefix;
@@ -473,125 +494,137 @@ __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, 
       if (in) atomicOr(&flags[t >> 5], 1u << (t & 31));
     }
     kdyn = kcap;
-    cluster.sync();   // pub_cnt may be written again
-  } else if (kcap > 0) {
-    for (int t = tid; t < n; t += NT) atomicOr(&flags[t >> 5], 1u << (t & 31));
-    kdyn = nC;
+  } else {
+    cluster.sync();   // the local maxima are visible
+    cluster_max();
+    if (kcap > 0) {
+      for (int t = tid; t < n; t += NT) atomicOr(&flags[t >> 5], 1u << (t & 31));
+      kdyn = nC;
+    }
   }
   __syncthreads();
 
-  // ---- 3. top-p cut inside the kcap winners ------------------------------------
+  // ---- 3. masses and winner counts, exchanged in one step ------------------------
+  // Z = sum of exp(S - M) over the candidates and W = the same over the kcap winners
+  // (fp64, fixed reduction trees, ranks added in order). If W < p * Z no prefix of
+  // the winners reaches p and all of them are kept (the common case when K_max binds).
+  const double Md = static_cast<double>(M);
+  const bool all_inf = !(M > -INFINITY);
+  double zl = 0.0, wl = 0.0;
   if (need_mass) {
     double z = 0.0, wsum = 0.0;
-    const double Md = static_cast<double>(M);
-    const bool all_inf = !(M > -INFINITY);
     for (int t = seg0; t < seg1; ++t) {
       const float s = S[c0 + lo + t];
       const double m = all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
       z += m;
       if ((flags[t >> 5] >> (t & 31)) & 1u) wsum += m;
     }
-    const double zl = block_allreduce<NT>(z, dscr, [](double x, double y) { return x + y; });
-    const double wl = block_allreduce<NT>(wsum, dscr, [](double x, double y) { return x + y; });
-    if (tid == 0) {
-      pub_z = zl;
-      pub_w = wl;
-    }
-    cluster.sync();
-    double Z = 0.0, W = 0.0;
-    for (int r = 0; r < CL; ++r) {
-      Z += *cluster.map_shared_rank(&pub_z, r);
-      W += *cluster.map_shared_rank(&pub_w, r);
-    }
-    if (!(W < static_cast<double>(ph) * Z)) {
-      // the cut may fall inside the winners: rank 0 orders all of them
-      int nsel = 0;
-      for (int t = seg0; t < seg1; ++t) nsel += (flags[t >> 5] >> (t & 31)) & 1u;
-      int tot;
-      int pos = block_exscan<NT>(nsel, s_iscr, tot);
-      for (int t = seg0; t < seg1; ++t)
-        if ((flags[t >> 5] >> (t & 31)) & 1u)
-          wbuf[pos++] = (static_cast<uint64_t>(keys[skew(t)]) << 32) | static_cast<uint32_t>(lo + t);
-      if (tid == 0) pub_cnt = tot;
-      cluster.sync();
-      if (rank == 0) {
-        int off = 0;
-        for (int r = 0; r < CL; ++r) {
-          const int cr = *cluster.map_shared_rank(&pub_cnt, r);
-          const uint64_t* src = cluster.map_shared_rank(wbuf, r);
-          for (int x = tid; x < cr; x += NT) sbuf[off + x] = src[x];
-          off += cr;
-        }
-        for (int x = off + tid; x < sort_n; x += NT) sbuf[x] = ~0ull;
-        __syncthreads();
-        for (int kk = 2; kk <= sort_n; kk <<= 1) {
-          for (int j = kk >> 1; j > 0; j >>= 1) {
-            for (int x = tid; x < sort_n; x += NT) {
-              const int y = x ^ j;
-              if (y > x) {
-                const uint64_t u = sbuf[x], v = sbuf[y];
-                const bool asc = (x & kk) == 0;
-                if ((u > v) == asc) {
-                  sbuf[x] = v;
-                  sbuf[y] = u;
-                }
-              }
-            }
-            __syncthreads();
-          }
-        }
-        const int E2 = (kdyn + NT - 1) / NT;
-        const int q0 = min(kdyn, tid * E2), q1 = min(kdyn, q0 + E2);
-        double loc = 0.0;
-        for (int x = q0; x < q1; ++x) {
-          const float s = S[c0 + static_cast<int>(sbuf[x] & 0xffffffffu)];
-          loc += all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
-        }
-        double dtot;
-        double run = block_exscan<NT>(loc, dscr, dtot);
-        if (tid == 0) s_hit = 0x7fffffff;
-        __syncthreads();
-        const double target = static_cast<double>(ph) * Z;
-        for (int x = q0; x < q1; ++x) {
-          const float s = S[c0 + static_cast<int>(sbuf[x] & 0xffffffffu)];
-          run += all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
-          if (run >= target) {
-            atomicMin(&s_hit, x);
-            break;
-          }
-        }
-        __syncthreads();
-        const int capC = min(a.k_max, nC);
-        if (tid == 0) pub_k = (s_hit != 0x7fffffff) ? max(min(s_hit + 1, capC), kminC) : kdyn;
-      }
-      cluster.sync();
-      const int k = *cluster.map_shared_rank(&pub_k, 0);
-      for (int w = tid; w < nflag_words; w += NT) flags[w] = 0u;
-      __syncthreads();
-      const uint64_t* order = cluster.map_shared_rank(sbuf, 0);
-      for (int x = tid; x < k; x += NT) {
-        const int id = static_cast<int>(order[x] & 0xffffffffu);
-        if (id >= lo && id < hi) atomicOr(&flags[(id - lo) >> 5], 1u << ((id - lo) & 31));
-      }
-      kdyn = k;
-      cluster.sync();   // rank 0's order is no longer read; pub_cnt may be written again
-    }
+    zl = block_allreduce<NT>(z, dscr, [](double x, double y) { return x + y; });
+    wl = block_allreduce<NT>(wsum, dscr, [](double x, double y) { return x + y; });
   }
-  __syncthreads();
-
-  // ---- 4. kept list: each CTA's ids after those of the lower ranks ----------------
   int nsel = 0;
   for (int t = seg0; t < seg1; ++t) nsel += (flags[t >> 5] >> (t & 31)) & 1u;
   int tot;
   int pos = block_exscan<NT>(nsel, s_iscr, tot);
-  if (tid == 0) pub_cnt = tot;
-  cluster.sync();
-  int below = 0, all = 0;
-  for (int r = 0; r < CL; ++r) {
-    const int v = *cluster.map_shared_rank(&pub_cnt, r);
-    if (r < rank) below += v;
-    all += v;
+  if (tid < CL) {
+    *cluster.map_shared_rank(&rx_z[rank], tid) = zl;
+    *cluster.map_shared_rank(&rx_w[rank], tid) = wl;
+    *cluster.map_shared_rank(&rx_sel[rank], tid) = tot;
   }
+  cluster.sync();
+  double Z = 0.0, W = 0.0;
+  int below = 0, all = 0;
+  for (int r = 0; r < CL; ++r) {   // rank order: a fixed summation order
+    Z += rx_z[r];
+    W += rx_w[r];
+    if (r < rank) below += rx_sel[r];
+    all += rx_sel[r];
+  }
+  if (need_mass && !(W < static_cast<double>(ph) * Z)) {
+    // the cut may fall inside the winners: rank 0 orders all of them
+    int wpos = pos;
+    for (int t = seg0; t < seg1; ++t)
+      if ((flags[t >> 5] >> (t & 31)) & 1u)
+        wbuf[wpos++] = (static_cast<uint64_t>(keys[skew(t)]) << 32) | static_cast<uint32_t>(lo + t);
+    if (tid == 0) pub_cnt = tot;
+    cluster.sync();
+    if (rank == 0) {
+      int off = 0;
+      for (int r = 0; r < CL; ++r) {
+        const int cr = *cluster.map_shared_rank(&pub_cnt, r);
+        const uint64_t* src = cluster.map_shared_rank(wbuf, r);
+        for (int x = tid; x < cr; x += NT) sbuf[off + x] = src[x];
+        off += cr;
+      }
+      for (int x = off + tid; x < sort_n; x += NT) sbuf[x] = ~0ull;
+      __syncthreads();
+      for (int kk = 2; kk <= sort_n; kk <<= 1) {
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+          for (int x = tid; x < sort_n; x += NT) {
+            const int y = x ^ j;
+            if (y > x) {
+              const uint64_t u = sbuf[x], v = sbuf[y];
+              const bool asc = (x & kk) == 0;
+              if ((u > v) == asc) {
+                sbuf[x] = v;
+                sbuf[y] = u;
+              }
+            }
+          }
+          __syncthreads();
+        }
+      }
+      const int E2 = (kdyn + NT - 1) / NT;
+      const int q0 = min(kdyn, tid * E2), q1 = min(kdyn, q0 + E2);
+      double loc = 0.0;
+      for (int x = q0; x < q1; ++x) {
+        const float s = S[c0 + static_cast<int>(sbuf[x] & 0xffffffffu)];
+        loc += all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
+      }
+      double dtot;
+      double run = block_exscan<NT>(loc, dscr, dtot);
+      if (tid == 0) s_hit = 0x7fffffff;
+      __syncthreads();
+      const double target = static_cast<double>(ph) * Z;
+      for (int x = q0; x < q1; ++x) {
+        const float s = S[c0 + static_cast<int>(sbuf[x] & 0xffffffffu)];
+        run += all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
+        if (run >= target) {
+          atomicMin(&s_hit, x);
+          break;
+        }
+      }
+      __syncthreads();
+      const int capC = min(a.k_max, nC);
+      if (tid == 0) pub_k = (s_hit != 0x7fffffff) ? max(min(s_hit + 1, capC), kminC) : kdyn;
+    }
+    cluster.sync();
+    const int k = *cluster.map_shared_rank(&pub_k, 0);
+    for (int w = tid; w < nflag_words; w += NT) flags[w] = 0u;
+    __syncthreads();
+    const uint64_t* order = cluster.map_shared_rank(sbuf, 0);
+    for (int x = tid; x < k; x += NT) {
+      const int id = static_cast<int>(order[x] & 0xffffffffu);
+      if (id >= lo && id < hi) atomicOr(&flags[(id - lo) >> 5], 1u << ((id - lo) & 31));
+    }
+    kdyn = k;
+    cluster.sync();   // every flag is set; rank 0's order is no longer read
+    // counts of the new winners
+    nsel = 0;
+    for (int t = seg0; t < seg1; ++t) nsel += (flags[t >> 5] >> (t & 31)) & 1u;
+    pos = block_exscan<NT>(nsel, s_iscr, tot);
+    if (tid == 0) pub_cnt = tot;
+    cluster.sync();
+    below = 0;
+    all = 0;
+    for (int r = 0; r < CL; ++r) {
+      const int v = *cluster.map_shared_rank(&pub_cnt, r);
+      if (r < rank) below += v;
+      all += v;
+    }
+  }
+
+  // ---- 4. kept list: each CTA's ids after those of the lower ranks ----------------
   for (int t = seg0; t < seg1; ++t)
     if ((flags[t >> 5] >> (t & 31)) & 1u) kept[c0 + below + pos++] = c0 + lo + t;
   if (rank == 0) {
@@ -674,8 +707,7 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   max_nc = max(max_nc, 1);
   if (a.phase == BSA_PHASE_DECODE && max_nc > 2048) {
     // few long rows: one cluster of CTAs per row
-    return max_nc <= 16384 ? launch_cluster<256>(a, rows, max_nc, s)
-                           : launch_cluster<512>(a, rows, max_nc, s);
+    return launch_cluster<256>(a, rows, max_nc, s);
   }
   if (max_nc <= 2048) return launch_nt<256>(a, rows, max_nc, s);
   if (max_nc <= 8192) return launch_nt<512>(a, rows, max_nc, s);
