@@ -388,6 +388,47 @@ def caches_for(inputs: dict):
     return k_idx, contiguous_cache(inputs["K"]), contiguous_cache(inputs["V"])
 
 
+class DecodeGraph:
+    """One decode step from host buffers as a single CUDA graph launch.
+
+    The graph holds, on fixed device buffers: the copy of the new query (q, q_idx)
+    from pinned host tensors, score -> select -> attend (the kernels keep their
+    programmatic dependent-launch edges), and the copy of o and lse back into pinned
+    host tensors. New queries are written into ``q_host`` / ``q_idx_host`` in place;
+    ``launch`` enqueues the step, ``run`` also waits for the host outputs."""
+
+    def __init__(self, step: DecodeStep, q_host, q_idx_host, k_idx, k: Cache, v: Cache,
+                 o_host, lse_host):
+        self.step, self.k_idx, self.k, self.v = step, k_idx, k, v
+        self.q_host, self.q_idx_host, self.o_host, self.lse_host = q_host, q_idx_host, o_host, lse_host
+        self.q_dev = torch.empty(q_host.shape, dtype=q_host.dtype, device="cuda")
+        self.q_idx_dev = torch.empty(q_idx_host.shape, dtype=q_idx_host.dtype, device="cuda")
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self._body()          # first launches (function attributes, tensor maps) uncaptured
+        side.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        # "relaxed": the entry points set kernel attributes on the host while capturing
+        with torch.cuda.graph(self.graph, capture_error_mode="relaxed"):
+            self._body()
+        torch.cuda.synchronize()
+
+    def _body(self):
+        self.q_dev.copy_(self.q_host, non_blocking=True)
+        self.q_idx_dev.copy_(self.q_idx_host, non_blocking=True)
+        self.step.run(self.q_dev, self.q_idx_dev, self.k_idx, self.k, self.v)
+        self.o_host.copy_(self.step.o, non_blocking=True)
+        self.lse_host.copy_(self.step.lse, non_blocking=True)
+
+    def launch(self):
+        self.graph.replay()
+
+    def run(self):
+        self.graph.replay()
+        torch.cuda.current_stream().synchronize()
+
+
 def decode_step_host(step: DecodeStep, q_host, q_idx_host, k_idx, k: Cache, v: Cache,
                      o_host, lse_host, q_dev=None, q_idx_dev=None, stream=None):
     """One decode step from host buffers: copy the new query (q, q_idx; pinned host

@@ -162,3 +162,35 @@ def test_decode_long_rows_cluster_select(p, k_min):
     x = W.make_decode_inputs(w, "cpu")
     step = run_decode(w, to_dev(x))
     parity.compare_decode_rows(w, x, step, all_rows(w))
+
+
+@pytest.mark.parametrize("name", ["decode_tiny_b1_h8_t4k", "decode_b8_h32_t32k_paged"])
+def test_decode_graph_matches_eager_and_oracle(name):
+    """The whole host-to-host decode step as one CUDA graph launch gives the same
+    bytes as the eager entry points, for the captured query and for a new query
+    written into the same pinned buffers; the replayed result also passes parity."""
+    w = W.WORKLOADS[name]
+    x = W.make_decode_inputs(w, "cpu")
+    xd = to_dev(x)
+    prob = bsa.problem_for(w, seq_lens=xd["seq_lens"], head_w=xd["head_w"])
+    k_idx, K, V = bsa.caches_for(xd)
+    q_h, qi_h = x["q"].clone().pin_memory(), x["q_idx"].clone().pin_memory()
+    eager = bsa.DecodeStep(prob)
+    graphed = bsa.DecodeStep(prob)
+    o_h = torch.empty(eager.o.shape, dtype=eager.o.dtype).pin_memory()
+    lse_h = torch.empty(eager.lse.shape, dtype=eager.lse.dtype).pin_memory()
+    g = bsa.DecodeGraph(graphed, q_h, qi_h, k_idx, K, V, o_h, lse_h)
+    for trial in range(2):
+        if trial == 1:   # a new query, written in place
+            gen = torch.Generator().manual_seed(5)
+            q_h.copy_(torch.randn(q_h.shape, generator=gen).to(q_h.dtype))
+            qi_h.copy_(torch.randn(qi_h.shape, generator=gen).to(qi_h.dtype))
+        eager.run(q_h.cuda(), qi_h.cuda(), k_idx, K, V)
+        g.run()
+        torch.cuda.synchronize()
+        assert int(eager.status.item()) == 0 and int(graphed.status.item()) == 0
+        assert torch.equal(o_h, eager.o.cpu())
+        assert torch.equal(lse_h, eager.lse.cpu())
+        assert torch.equal(graphed.kept.cpu(), eager.kept.cpu())
+    x2 = dict(x, q=q_h.clone(), q_idx=qi_h.clone())
+    parity.compare_decode_rows(w, x2, graphed, all_rows(w)[:4])
