@@ -14,6 +14,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import math
 import os
 import statistics
@@ -48,10 +49,15 @@ def load_peaks():
 
 
 def kernel_source_hash(files):
+    """Hash of the kernel sources with comments and whitespace removed, so that a
+    comment edit does not void a measurement taken on the same code."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "block_sparse_long_06_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "block_sparse_long_06_b200", "csrc", f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(re.sub(r"\s+", "", text).encode())
     return h.hexdigest()[:16]
 
 

@@ -16,9 +16,9 @@
 //    into one stage of a K/V ring (TMA, 128-byte swizzle);
 //  * three MMA-issuing threads (warps 1-2: scores of tile 0/1, warp 3: P.V of both
 //    tiles): a single thread can issue a tcgen05.mma only every ~50 cycles and a
-//    commit costs about as much, so one issuer would leave the tensor core idle. S_t(j) = Q_t K_j^T (bf16, M = 128,
-//    N = 64, K = d) goes to one of the tile's two S buffers in tensor memory;
-//    O_t += P_t(j) V_j (fp16, P read from tensor memory over the S columns, N = d).
+//    commit costs about as much, so one issuer would leave the tensor core idle.
+//    S_t(j) = Q_t K_j^T (bf16, M = 128, N = 64, K = d) goes to the tile's S buffer in
+//    tensor memory; O_t += P_t(j) V_j (fp16, P read from tensor memory, N = d).
 //    P has tensor-memory buffers of its own (two per tile), so the S buffer of a
 //    tile is free as soon as its softmax warps have loaded S into registers: the
 //    score MMAs of step j+1 run while the softmax of step j computes, and the P.V

@@ -28,7 +28,10 @@
 // tokens) run on a cluster of up to 8 CTAs per row: each CTA holds a contiguous
 // slice of the candidates, and the cluster combines its maxima, radix histograms,
 // equal-key counts, masses and output offsets through distributed shared memory,
-// always in rank order, so every CTA takes the same decisions.
+// always in rank order, so every CTA takes the same decisions. Each CTA pushes its
+// values into every peer's shared memory before a cluster barrier (remote stores do
+// not stall; remote loads would wait about a thousand cycles each), and the common
+// path needs one barrier per radix pass plus three.
 #include <cooperative_groups.h>
 
 #include "bsa_common.cuh"
