@@ -242,7 +242,10 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def one_step(ev=None):
+    def one_step(ev=None, split=False, prefill=True):
+        """One step. split=True also records an event between selection and attention
+        (to time bsa_decode alone); it is left out of the step timing because an event
+        there keeps the attention kernel from overlapping the selection's tail."""
         if do_dec:
             flush.zero_()                   # L2 flushed between decode steps (untimed)
         if ev:
@@ -253,13 +256,15 @@ def run_ours(args, world, rank, local):
             else:
                 bsa.bsa_score_blocks(dprob, xd["q_idx"], k_idx_c, dstep.scores, dstep.status)
             bsa.bsa_select_top_p(dprob, dstep.scores, dstep.kept, dstep.kept_count, dstep.status)
-        if ev:
+        if ev and split:
             ev["a0"].record(stream)
         if do_dec:
             bsa.bsa_decode(dprob, xd["q"], K_c, V_c, dstep.kept, dstep.kept_count, dstep.o,
                            dstep.lse, None, dstep.workspace, dstep.status)
         if ev:
             ev["d1"].record(stream)
+        if not prefill:
+            return
         if do_pf:
             flush.zero_()                   # and before the prefill (its inputs fit in L2)
         if ev:
@@ -282,6 +287,7 @@ def run_ours(args, world, rank, local):
 
     names = ("d0", "a0", "d1", "p0", "p1", "p2")
     evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
+    evs_att = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device() if world == 1 else local) as clk:
@@ -291,10 +297,13 @@ def run_ours(args, world, rank, local):
         for k in range(args.steps):
             one_step(evs[k])
         t_end.record(stream)
+        if do_dec:                          # bsa_decode alone: the same steps, split timing
+            for k in range(args.steps):
+                one_step(evs_att[k], split=True, prefill=False)
         torch.cuda.synchronize()
     barrier(world)
     dec_ms = [e["d0"].elapsed_time(e["d1"]) for e in evs]
-    att_ms = [e["a0"].elapsed_time(e["d1"]) for e in evs]
+    att_ms = [e["a0"].elapsed_time(e["d1"]) for e in evs_att] if do_dec else [0.0] * args.steps
     psel_ms = [e["p0"].elapsed_time(e["p1"]) for e in evs]
     patt_ms = [e["p1"].elapsed_time(e["p2"]) for e in evs]
     total_ms = t_start.elapsed_time(t_end)
@@ -363,8 +372,9 @@ def run_ours(args, world, rank, local):
                     "outside the timed events")
     config["parallelism"] = f"dp{world} (independent sequences per GPU)"
     # kernels per step: decode = scorer, selection, split-K attention, LSE merge;
-    # prefill = scorer, selection, V->fp16, attention
-    launches = args.steps * (4 * do_dec + 4 * do_pf)
+    # prefill = scorer, selection, V->fp16, attention; then the decode-only steps
+    # that time bsa_decode alone
+    launches = args.steps * (4 * do_dec + 4 * do_pf) + args.steps * 4 * do_dec
     if do_dec:
         value, unit = dec["tokens_per_s"], "tokens/s"
     else:
