@@ -52,8 +52,53 @@ BSA_DEVFN uint32_t order_key(float s) {
   u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending in s
   return ~u;                                  // ascending key = descending score
 }
+// The score of a key (exact; -0 comes back as +0 and NaN as a NaN), so the mass
+// sums read the keys already in shared memory instead of the scores in global memory.
+BSA_DEVFN float key_score(uint32_t key) {
+  const uint32_t u = ~key;
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
 
 __host__ __device__ __forceinline__ int skew(int i) { return i + (i >> 5); }
+
+// Keys of the scores S[0, n) into shared memory; returns this thread's max score. The
+// loads of 8 rounds are issued before any is used (one dependent round trip to L2
+// each would dominate the selection of a short row).
+template <int NT>
+BSA_DEVFN float load_keys(const float* S, int n, uint32_t* keys, int tid) {
+  float lmax = -INFINITY;
+  for (int t0 = 0; t0 < n; t0 += 8 * NT) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = t0 + u * NT + tid;
+      v[u] = t < n ? S[t] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int t = t0 + u * NT + tid;
+      if (t < n) {
+        keys[skew(t)] = order_key(v[u]);
+        if (v[u] == v[u]) lmax = fmaxf(lmax, v[u]);
+      }
+    }
+  }
+  return lmax;
+}
+
+// Adds the digit of one key to a shared-memory histogram. Pass 0 reads the top byte,
+// which most keys share: equal digits of a warp are combined first (match.any). In
+// later passes the digits are spread out and match.any would cost more than it
+// saves (it was a third of a 128K row's selection), so each lane adds its own.
+BSA_DEVFN void hist_add(uint32_t* h, uint32_t digit, int pass, int lane) {
+  if (pass == 0) {
+    const uint32_t peers = __match_any_sync(0xffffffffu, digit);
+    if (digit < 256u && lane == __ffs(peers) - 1) atomicAdd(&h[digit], __popc(peers));
+  } else if (digit < 256u) {
+    atomicAdd(&h[digit], 1u);
+  }
+}
 
 // Deterministic block reductions / scans (fixed tree for a fixed NT).
 template <int NT, typename T, typename Op>
@@ -149,12 +194,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_
   const bool need_mass = (ph > 0.f) && (ph < 1.f) && kcap > 0;
 
   // ---- 1. keys and max ------------------------------------------------------
-  float lmax = -INFINITY;
-  for (int t = tid; t < nC; t += NT) {
-    const float s = S[c0 + t];
-    keys[skew(t)] = order_key(s);
-    if (s == s) lmax = fmaxf(lmax, s);
-  }
+  const float lmax = load_keys<NT>(S + c0, nC, keys, tid);
   for (int w = tid; w < nflag_words; w += NT) flags[w] = 0u;
   const float M = block_allreduce<NT>(lmax, s_fscr, [](float x, float y) { return fmaxf(x, y); });
 
@@ -179,8 +219,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_
           const uint32_t k = keys[skew(t)];
           if ((k & pmask) == prefix) digit = (k >> shift) & 255u;
         }
-        const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-        if (digit < 256u && lane == __ffs(peers) - 1) atomicAdd(&h[digit], __popc(peers));
+        hist_add(h, digit, pass, lane);
       }
       __syncthreads();
       for (int x = tid; x < 256; x += NT) {
@@ -246,7 +285,7 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_
     const double Md = static_cast<double>(M);
     const bool all_inf = !(M > -INFINITY);
     for (int t = seg0; t < seg1; ++t) {
-      const float s = S[c0 + t];
+      const float s = key_score(keys[skew(t)]);
       const double m = all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
       z += m;
       if ((flags[t >> 5] >> (t & 31)) & 1u) wsum += m;
@@ -396,12 +435,7 @@ __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, 
   const int lo = min(nC, rank * per_cta), hi = min(nC, lo + per_cta), n = hi - lo;
 
   // ---- 1. keys and the local max (published with the first exchange) -----------
-  float lmax = -INFINITY;
-  for (int t = tid; t < n; t += NT) {
-    const float s = S[c0 + lo + t];
-    keys[skew(t)] = order_key(s);
-    if (s == s) lmax = fmaxf(lmax, s);
-  }
+  float lmax = load_keys<NT>(S + c0 + lo, n, keys, tid);
   for (int w = tid; w < nflag_words; w += NT) flags[w] = 0u;
   lmax = block_allreduce<NT>(lmax, s_fscr, [](float x, float y) { return fmaxf(x, y); });
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
@@ -433,8 +467,7 @@ __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, 
           const uint32_t k = keys[skew(t)];
           if ((k & pmask) == prefix) digit = (k >> shift) & 255u;
         }
-        const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-        if (digit < 256u && lane == __ffs(peers) - 1) atomicAdd(&h[digit], __popc(peers));
+        hist_add(h, digit, pass, lane);
       }
       __syncthreads();
       for (int x = tid; x < 256; x += NT) {
@@ -517,7 +550,7 @@ __global__ void __launch_bounds__(NT) select_cluster_kernel(const SelectArgs a, 
   if (need_mass) {
     double z = 0.0, wsum = 0.0;
     for (int t = seg0; t < seg1; ++t) {
-      const float s = S[c0 + lo + t];
+      const float s = key_score(keys[skew(t)]);
       const double m = all_inf ? 1.0 : ((s == s) ? exp(static_cast<double>(s) - Md) : 0.0);
       z += m;
       if ((flags[t >> 5] >> (t & 31)) & 1u) wsum += m;
