@@ -4,8 +4,8 @@ This module only draws inputs: random tensors, planted heavy-hitter keys, page
 tables. It holds none of the method's arithmetic (no scoring, selection or
 attention), so both the CUDA path and the fp64 oracle can consume its output.
 
-Recipe (the pages give workload shapes in prose only; the readings are listed in
-DESIGN.md):
+Recipe (the pages give workload shapes in prose only; where they leave a detail
+open, the plainest reading is taken and stated here):
 * Q, K, V ~ N(0, 1), stored bf16.
 * One shared index projection W_idx [d, r] ~ N(0, 1/d); index keys
   k_idx = bf16(K_bf16 @ W_idx), index queries q_idx = bf16(Q_bf16 @ W_idx).

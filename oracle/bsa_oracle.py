@@ -30,7 +30,7 @@ Sources (gist.science technical summaries; cited by page title and section):
   (PBS-Attn), Methodology §1: attention output is invariant to permuting
   key/value pairs (used by the tests as an invariant).
 
-Readings where the pages leave a step open (each also listed in the design doc):
+Readings where the pages leave a step open:
 
 * block aggregate of token scores = max over the block's tokens (and, in
   prefill, over the query block's tokens too);
@@ -95,10 +95,7 @@ def token_scores(q_idx_heads: np.ndarray, k_idx_tokens: np.ndarray, head_w: np.n
     k_idx_tokens: [n_k, r].  head_w: [G].
     Returns [n_k] or [n_q, n_k].
     """
-    if q_idx_heads.ndim == 2:
-        dots = q_idx_heads @ k_idx_tokens.T                      # [G, n_k]
-        return idx_scale * np.tensordot(head_w, np.maximum(dots, 0.0), axes=(0, 0))
-    dots = np.einsum("gqr,kr->gqk", q_idx_heads, k_idx_tokens)  # [G, n_q, n_k]
+    dots = q_idx_heads @ k_idx_tokens.T                  # [G, n_k] or [G, n_q, n_k]
     return idx_scale * np.tensordot(head_w, np.maximum(dots, 0.0), axes=(0, 0))
 
 

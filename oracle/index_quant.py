@@ -8,7 +8,7 @@ from the product.
 Source: SpotAttention, Methodology §4 "quantisation": the selector's K cache
 (the index keys) may be stored as microscaled INT4 or FP4, about 3.5x smaller
 than bf16, while the backbone's K/V cache stays untouched. The page names the
-idea and the ratio, not the format. Reading (also listed in the design doc):
+idea and the ratio, not the format. Reading:
 
 * a micro-block is one token's r = 16 index-key elements; it carries one FP8
   E4M3 scale (4 + 8/16 = 4.5 bits per element, 32 B -> 9 B per token = 3.56x,
