@@ -36,6 +36,8 @@ METRIC = "decode tokens/s & achieved HBM GB/s at 128K ctx; sparse-prefill TFLOP/
 DECODE_WL = "decode_b32_h32_t128k_paged"
 PREFILL_WL = "prefill_b1_h32_t64k"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures (HGX): 7.7 TB/s HBM3e, 2.25 PFLOP/s dense bf16
+DATASHEET = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
 
 
 # ---------------------------------------------------------------- helpers
@@ -46,6 +48,15 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def peak_clock_note(peaks):
+    """The SM clock the measured matmul peak was taken at, when the peaks file says."""
+    c = peaks.get("clocks_under_load") or {}
+    if c.get("sm_mhz_median"):
+        return (f"measured peak taken at a median SM clock of {c['sm_mhz_median']:.0f} MHz "
+                f"(max {c.get('sm_max_mhz', 0):.0f} MHz)")
+    return None
 
 
 def kernel_source_hash(files):
@@ -190,8 +201,17 @@ def decode_bytes(w, kept_count, seq_lens, index_cache="bf16"):
 
 
 def prefill_flops(w, kept_count):
-    kc = kept_count.to(torch.int64).cpu()
-    return float(kc.sum()) * w.G * 4 * 64 * 64 * w.d
+    """(kept-tile FLOP, causal-exact FLOP) of one prefill. The first counts every kept
+    64 x 64 tile whole, as the tensor cores compute it (the headline: FLOPs of the
+    kept tiles); the second counts only the (query, key) pairs the causal mask leaves
+    visible: half of each diagonal tile plus its diagonal, and the real rows of a
+    partial last query block."""
+    kc = kept_count.to(torch.int64).cpu().reshape(-1, w.nb)    # [B*Hkv, nqb]
+    tiles = float(kc.sum()) * w.G * 4 * 64 * 64 * w.d
+    nq = torch.tensor([min(64, w.T - 64 * i) for i in range(w.nb)], dtype=torch.int64)
+    # every kept block but the diagonal is fully visible to the block's real rows
+    pairs = ((kc - 1).clamp(min=0) * nq * 64).sum() + (nq * (nq + 1) // 2).sum() * kc.shape[0]
+    return tiles, float(pairs) * w.G * 4 * w.d
 
 
 # ---------------------------------------------------------------- our arm
@@ -333,20 +353,27 @@ def run_ours(args, world, rank, local):
         files = ["decode_attn.cu", "bsa_common.cuh", "bsa_internal.h"]
         roof_dec = {"bound": "hbm", "kernel": "bsa_decode (split-K attention + LSE merge)",
                     "achieved": attn_gbs, "peak": hbm, "unit": "GB/s", "frac": attn_gbs / hbm,
+                    "peak_datasheet": DATASHEET["hbm_gbs"],
+                    "frac_datasheet": attn_gbs / DATASHEET["hbm_gbs"],
                     "traffic": ncu_traffic("decode_attn", files, wd.name),
                     "peak_source": f"{peak_src} hbm_gbs (burst copy)",
                     "bytes_per_launch": by["attention"]}
     if do_pf:
-        flops = prefill_flops(wp, pf.kept_count)
+        flops, flops_exact = prefill_flops(wp, pf.kept_count)
         patt_avg = max(patt_avg, 1e-9)
         pf_tflops = world * flops / (patt_avg / 1e3) / 1e12
         pre = {"select_ms": psel_avg, "attention_ms": patt_avg, "tflops": pf_tflops,
-               "tensor_frac": pf_tflops / world / tflops_peak, "kept_tile_flop": flops}
-        files = ["prefill_tc.cu", "prefill_attn.cu", "tcgen05.cuh", "bsa_common.cuh",
+               "tensor_frac": pf_tflops / world / tflops_peak, "kept_tile_flop": flops,
+               "causal_exact_flop": flops_exact,
+               "causal_exact_tflops": world * flops_exact / (patt_avg / 1e3) / 1e12}
+        files = ["prefill_tc.cu", "v_to_f16.cu", "tcgen05.cuh", "bsa_common.cuh",
                  "bsa_internal.h"]
         roof_pf = {"bound": "tensor", "kernel": "bsa_prefill (V->fp16 + attention)",
                    "achieved": pf_tflops / world, "peak": tflops_peak, "unit": "TFLOP/s",
                    "frac": pf_tflops / world / tflops_peak,
+                   "peak_datasheet": DATASHEET["bf16_tflops"],
+                   "frac_datasheet": pf_tflops / world / DATASHEET["bf16_tflops"],
+                   "peak_clock": peak_clock_note(peaks),
                    "traffic": ncu_traffic("prefill_tc", files, wp.name),
                    "peak_source": f"{peak_src} bf16_tflops (burst)",
                    "flop_per_launch": flops}
@@ -448,13 +475,15 @@ def run_e2e(args, dprob, dstep, xd, k_idx_c, K_c, V_c, stream, world):
 
 
 # ---------------------------------------------------------------- oracle on the host
-def blas_threads():
+def one_thread():
+    """Context in which the oracle runs on one host thread (numpy's BLAS pools limited
+    to 1), so the reported core count is the number of threads that actually worked."""
+    import contextlib
     try:
-        from threadpoolctl import threadpool_info
-        n = [p.get("num_threads", 1) for p in threadpool_info()]
-        return max(n) if n else 1
-    except Exception:
-        return 1
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=1)
+    except ImportError:
+        return contextlib.nullcontext()
 
 
 def cpu_baseline_decode(w, xd, dstep=None, budget_s=20.0, max_seqs=None):
@@ -478,22 +507,23 @@ def cpu_baseline_decode(w, xd, dstep=None, budget_s=20.0, max_seqs=None):
             Kb = xd["K"][pages].transpose(0, 1).reshape(w.Hkv, -1, w.d)[:, :T].cpu()
             Vb = xd["V"][pages].transpose(0, 1).reshape(w.Hkv, -1, w.d)[:, :T].cpu()
         hw = xd["head_w"].double().cpu().numpy()
-        t0 = time.perf_counter()
-        for g in range(w.Hkv):
-            S = O.decode_block_scores(qi[g * G:(g + 1) * G].double().numpy(),
-                                      ki[g, :T].double().numpy(), T, hw[g * G:(g + 1) * G],
-                                      1.0 / math.sqrt(w.r))
-            sel = O.select_decode(S, w.n_sink, w.n_local, w.p, w.k_max, w.k_min)
-            ids = O.kept_token_ids(sel.kept, T)
-            O.attend(q[g * G:(g + 1) * G].double().numpy(), Kb[g, ids].double().numpy(),
-                     Vb[g, ids].double().numpy(), 1.0 / math.sqrt(w.d))
-        t_total += time.perf_counter() - t0
+        with one_thread():
+            t0 = time.perf_counter()
+            for g in range(w.Hkv):
+                S = O.decode_block_scores(qi[g * G:(g + 1) * G].double().numpy(),
+                                          ki[g, :T].double().numpy(), T, hw[g * G:(g + 1) * G],
+                                          1.0 / math.sqrt(w.r))
+                sel = O.select_decode(S, w.n_sink, w.n_local, w.p, w.k_max, w.k_min)
+                ids = O.kept_token_ids(sel.kept, T)
+                O.attend(q[g * G:(g + 1) * G].double().numpy(), Kb[g, ids].double().numpy(),
+                         Vb[g, ids].double().numpy(), 1.0 / math.sqrt(w.d))
+            t_total += time.perf_counter() - t0
         done_seqs += 1
         b += 1
         if t_total >= budget_s:
             break
-    return {"value": done_seqs / t_total, "unit": "tokens/s", "cores": blas_threads(),
-            "kind": "oracle",
+    return {"value": done_seqs / t_total, "unit": "tokens/s", "cores": 1,
+            "host_cores": os.cpu_count(), "kind": "oracle",
             "sample": f"{done_seqs} of {w.B} sequences of {w.name} (all {w.Hkv} kv heads each: "
                       f"score, select, attend in float64), {t_total:.1f} s"}
 
@@ -515,7 +545,8 @@ def run_reference(args, world, rank):
             per_step.append(1.0 / r["value"])     # seconds for one sequence
     sec = sum(per_step)
     value = args.steps / sec
-    cpu = {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+    cpu = {"value": value, "unit": "tokens/s", "cores": 1, "host_cores": os.cpu_count(),
+           "kind": "oracle",
            "sample": f"one sequence (all {wd.Hkv} kv heads) of {DECODE_WL} per step"}
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

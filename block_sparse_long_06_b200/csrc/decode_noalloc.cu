@@ -11,9 +11,13 @@
 // keeps until the process exits. Nothing here calls cudaMalloc, cudaFree or any
 // allocating routine.
 //
-// The first call on a device (with that device current) looks up the array's
-// device address with cudaGetSymbolAddress and remembers it; make that first
-// call before any stream capture. Every call on a device shares the one array,
+// Every call made outside stream capture looks up the array's device address
+// on the current device with cudaGetSymbolAddress and remembers it per device,
+// so a context that was reset and re-created gets its own address. A call whose
+// stream is capturing cannot make that lookup part of a graph and uses the
+// address remembered by the last uncaptured call on the device: make one call
+// before capturing (a capture with none returns BSA_ERR_UNSUPPORTED). Every call
+// on a device shares the one array,
 // so calls whose work overlaps on the GPU (different streams, or concurrent host
 // threads) race on it: serialise them. The array keeps whatever the last call
 // wrote; the decode kernels write every partial they later read, so nothing has
@@ -30,19 +34,25 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_decode_scratch on the current device (looked up once per device).
-bsa_status_t scratch_address(void** out) {
+// Device address of g_decode_scratch on the current device: looked up again on
+// every call outside stream capture, taken from the last lookup while capturing.
+bsa_status_t scratch_address(cudaStream_t stream, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return bsa::record_cuda_error(e);
   if (dev < 0 || dev >= kMaxDevices) return BSA_ERR_UNSUPPORTED;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(stream, &cs);
+  if (e != cudaSuccess) return bsa::record_cuda_error(e);
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (cs == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess || p == nullptr)
       return bsa::record_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
     g_scratch_addr[dev] = p;
+  } else if (g_scratch_addr[dev] == nullptr) {
+    return BSA_ERR_UNSUPPORTED;
   }
   *out = g_scratch_addr[dev];
   return BSA_OK;
@@ -59,7 +69,7 @@ extern "C" bsa_status_t bsa_decode_noalloc(const bsa_problem_t* prob, const void
   if (st != BSA_OK) return st;
   if (need > static_cast<size_t>(BSA_NOALLOC_SCRATCH_BYTES)) return BSA_ERR_WORKSPACE;
   void* scratch = nullptr;
-  if ((st = scratch_address(&scratch)) != BSA_OK) return st;
+  if ((st = scratch_address(static_cast<cudaStream_t>(stream), &scratch)) != BSA_OK) return st;
   return bsa_decode(prob, q, k, v, kept, kept_count, o, lse, o_f32, scratch,
                     static_cast<size_t>(BSA_NOALLOC_SCRATCH_BYTES), dev_status, stream);
 }

@@ -4,7 +4,9 @@
 // error well inside the tolerance) and an MMA takes both operands in one type,
 // so V is converted once from the bf16 cache into an fp16 copy in the workspace,
 // laid out [B*Hkv, Tpad, d] (Tpad = T rounded up to 64, zero padded). Values
-// outside the fp16 range are reported (BSA_DEV_FP16_RANGE).
+// outside the fp16 range are reported (BSA_DEV_FP16_RANGE); rows of a page id
+// outside the pool or past the cache extent are left zero and reported
+// (BSA_DEV_BAD_PAGE), as the attention kernel masks their keys.
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
 
@@ -16,7 +18,7 @@ __global__ void v_to_f16_kernel(const PrefillArgs a) {
   const int64_t nvec = static_cast<int64_t>(a.B) * a.Hkv * a.Tpad * (a.d / 8);
   const char* vbase = static_cast<const char*>(a.v.base);
   uint4* out = static_cast<uint4*>(const_cast<void*>(a.v16));
-  bool bad = false;
+  bool range_bad = false, page_bad = false;
   for (int64_t x = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; x < nvec;
        x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t vecs_per_row = a.d / 8;
@@ -45,17 +47,18 @@ __global__ void v_to_f16_kernel(const PrefillArgs a) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float2 f = unpack_bf16(w[q]);
-          if (fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f) bad = true;
+          if (fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f) range_bad = true;
           o4[q] = pack_f16(f.x, f.y);
         }
         res = make_uint4(o4[0], o4[1], o4[2], o4[3]);
       } else {
-        bad = true;
+        page_bad = true;
       }
     }
     out[x] = res;
   }
-  if (bad) report(a.status, BSA_DEV_FP16_RANGE);
+  if (range_bad) report(a.status, BSA_DEV_FP16_RANGE);
+  if (page_bad) report(a.status, BSA_DEV_BAD_PAGE);
 }
 
 }  // namespace

@@ -236,10 +236,13 @@ bsa_status_t bsa_score_blocks_q(const bsa_problem_t* prob, const void* q_idx, bs
  * Arguments and outputs are those of bsa_decode minus the workspace. Returns
  * BSA_ERR_WORKSPACE, launching nothing, when the problem needs more scratch than
  * BSA_NOALLOC_SCRATCH_BYTES (bsa_workspace_size(BSA_OP_DECODE) tells how much).
- * The first call on a device looks up the array's address (cudaGetSymbolAddress)
- * with that device current; make it before any stream capture. All calls on a
- * device share the array: calls whose work overlaps on the GPU race and must be
- * serialised by the caller. Allocates and frees nothing. */
+ * Every call outside stream capture looks up the array's address on the current
+ * device (cudaGetSymbolAddress), so a reset and re-created context is followed; a
+ * call on a capturing stream reuses the address of the last uncaptured call on
+ * that device and returns BSA_ERR_UNSUPPORTED when there was none, so make one
+ * call before capturing. All calls on a device share the array: calls whose work
+ * overlaps on the GPU race and must be serialised by the caller. Allocates and
+ * frees nothing. */
 bsa_status_t bsa_decode_noalloc(const bsa_problem_t* prob, const void* q, bsa_cache_t k,
                                 bsa_cache_t v, const int32_t* kept, const int32_t* kept_count,
                                 void* o, float* lse, float* o_f32, int32_t* dev_status,

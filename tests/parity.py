@@ -197,8 +197,26 @@ def oracle_prefill_rows(w, inputs, b, g, rows, kept_override=None):
                           rows=rows, kept_override=kept_override)
 
 
-def compare_prefill_rows(w, inputs, pf, b, g, rows, check_scores=True):
+def _check_prefill_block(w, o32, lse, b, g, i, ref, summary):
     G, T = w.G, w.T
+    q0, q1 = i * 64, min(i * 64 + 64, T)
+    o32_blk = o32[b, g * G:(g + 1) * G, q0:q1].double().numpy()
+    lse_blk = lse[b, g * G:(g + 1) * G, q0:q1].double().numpy()
+    errs = attention_errors(o32_blk, None, lse_blk, ref["o"], ref["lse"])
+    check_attention(errs, f"prefill row {(b, g, i)}")
+    for k_ in ("max_abs", "rel_l2", "lse_abs"):
+        summary[k_] = max(summary[k_], errs[k_])
+    summary["rows"] += 1
+
+
+def compare_prefill_rows(w, inputs, pf, b, g, rows, check_scores=True, kept_dev=None,
+                         attend_lists=None):
+    """Compare a finished Prefill with the oracle on query blocks ``rows`` of (b, g).
+
+    kept_dev: {i: list} kept lists the selection produced, when pf.kept was changed
+    afterwards (default: pf.kept). attend_lists: {i: list} kept lists the attention
+    is to be checked against (default: the selected set, or the device's set when
+    the tie rule accepted it)."""
     kept = pf.kept.cpu()
     cnt = pf.kept_count.cpu()
     scores = pf.scores.cpu()
@@ -208,31 +226,28 @@ def compare_prefill_rows(w, inputs, pf, b, g, rows, check_scores=True):
     summary = {"rows": 0, "ties": 0, "max_abs": 0.0, "rel_l2": 0.0, "lse_abs": 0.0,
                "score_rel": 0.0}
     refs = oracle_prefill_rows(w, inputs, b, g, rows)
-    override = {}
+    override = dict(attend_lists or {})
     for i, ref in refs.items():
         if i and check_scores:
             S_dev = scores[b, g, i, :i].double().numpy()
             rel = np.max(np.abs(S_dev - ref["S"]) / np.maximum(1.0, np.abs(ref["S"])))
             summary["score_rel"] = max(summary["score_rel"], float(rel))
             assert rel <= SCORE_REL, f"prefill row {(b, g, i)}: score rel err {rel}"
-        c = int(cnt[b, g, i])
-        kd = kept[b, g, i, :c].tolist()
-        assert all(x == -1 for x in kept[b, g, i, c:].tolist()), "padding is not -1"
+        if kept_dev is not None and i in kept_dev:
+            kd = list(kept_dev[i])
+        else:
+            c = int(cnt[b, g, i])
+            kd = kept[b, g, i, :c].tolist()
+            assert all(x == -1 for x in kept[b, g, i, c:].tolist()), "padding is not -1"
         verdict = selection_verdict(ref["sel"], kd, w.p)
         assert not verdict.startswith("mismatch"), f"prefill row {(b, g, i)}: {verdict}"
         if verdict == "tie":
             summary["ties"] += 1
-            override[i] = kd
+            override.setdefault(i, kd)
     if override:
         refs.update(oracle_prefill_rows(w, inputs, b, g, list(override), kept_override=override))
     for i, ref in refs.items():
-        q0, q1 = i * 64, min(i * 64 + 64, T)
-        o32_blk = o32[b, g * G:(g + 1) * G, q0:q1].double().numpy()
-        lse_blk = lse[b, g * G:(g + 1) * G, q0:q1].double().numpy()
-        errs = attention_errors(o32_blk, None, lse_blk, ref["o"], ref["lse"])
-        check_attention(errs, f"prefill row {(b, g, i)}")
-        for k_ in ("max_abs", "rel_l2", "lse_abs"):
-            summary[k_] = max(summary[k_], errs[k_])
-        summary["rows"] += 1
+        _check_prefill_block(w, o32, lse, b, g, i, ref, summary)
+    G = w.G
     assert bf16_is_rne_of_f32(o[b, g * G:(g + 1) * G], o32[b, g * G:(g + 1) * G])
     return summary

@@ -130,20 +130,17 @@ def test_bad_page_id_is_reported_not_trapped():
 
 
 # ---------------------------------------------------------------- full-size workloads
-FULL_ROWS = {
-    "decode_b8_h32_t32k_paged": [(0, 0), (1, 3), (3, 7), (7, 5)],
-    "decode_b32_h32_t128k_paged": [(0, 0), (1, 2), (16, 5), (31, 7)],
-    "decode_b1_h64_t1m": [(0, 0), (0, 3), (0, 7)],
-}
-
-
-@pytest.mark.parametrize("name", list(FULL_ROWS))
-def test_decode_full_size_sampled_rows(name):
+# Every row of every full-size decode workload: the 1M rows are the only inputs of
+# the cluster selection at full size (16,374 candidates per row).
+@pytest.mark.parametrize("name", ["decode_b8_h32_t32k_paged", "decode_b32_h32_t128k_paged",
+                                  "decode_b1_h64_t1m"])
+def test_decode_full_size_every_row(name):
     w = W.WORKLOADS[name]
     x = W.make_decode_inputs(w, "cuda")
     step = run_decode(w, x)
-    s = parity.compare_decode_rows(w, x, step, FULL_ROWS[name])
-    print(name, s)
+    s = parity.compare_decode_rows(w, x, step, all_rows(w))
+    print(f"{name}: {s['rows']} rows compared, {s['ties']} ties", s)
+    assert s["rows"] == w.B * w.Hkv
     # every row keeps sinks + local + at most k_max dynamic blocks
     assert int(step.kept_count.max()) <= w.n_sink + w.n_local + w.k_max
     del x, step

@@ -76,14 +76,23 @@ def test_prefill_top_p_and_kmin():
         parity.compare_prefill_rows(w, x, pf, 0, g, list(range(14)))
 
 
-def test_prefill_full_size_sampled_rows():
+def test_prefill_full_size_rows_of_every_kv_head():
+    """The 64K workload: every kv head on query blocks 0-3 (sinks and local windows
+    overlap the diagonal), 67-69 (where kept(i) = min(i + 1, 68) saturates), every
+    64th block and the last one."""
     w = W.WORKLOADS["prefill_b1_h32_t64k"]
     x = W.make_prefill_inputs(w, "cuda")
     pf = run_prefill(w, x)
-    rows = [0, 1, 2, 3, 66, 67, 68, 511, 1023]
-    for g in (0, 5):
+    rows = sorted({0, 1, 2, 3, 67, 68, 69, w.nb - 1} | set(range(64, w.nb, 64)))
+    total = {"rows": 0, "ties": 0}
+    for g in range(w.Hkv):
         s = parity.compare_prefill_rows(w, x, pf, 0, g, rows)
-        print("prefill full", g, s)
-    # kept(i) = min(i + 1, 68) for this configuration
-    kc = pf.kept_count[0, 0].cpu()
-    assert all(int(kc[i]) == min(i + 1, 68) for i in range(w.nb))
+        total["rows"] += s["rows"]
+        total["ties"] += s["ties"]
+        print("prefill 64K, kv head", g, s)
+    print(f"prefill 64K: {total['rows']} rows compared, {total['ties']} ties")
+    assert total["rows"] == w.Hkv * len(rows)
+    # kept(i) = min(i + 1, 68) for this configuration, on every row
+    kc = pf.kept_count[0].cpu()
+    expect = torch.tensor([min(i + 1, 68) for i in range(w.nb)], dtype=kc.dtype)
+    assert torch.equal(kc, expect.expand_as(kc))

@@ -6,11 +6,13 @@ device) get the decode attention step with its split-K scratch in the library's
 fixed device array instead of a workspace they would have to allocate. These
 tests call it through the C ABI and compare it with bsa_decode, which takes a
 caller-allocated workspace, on two calls in a row (the array keeps the previous
-call's contents, which must not leak into the next result).
+call's contents, which must not leak into the next result), and each call's
+output with the fp64 oracle on every row.
 
 This file is named to be collected last.
 """
 import ctypes
+from types import SimpleNamespace
 
 import pytest
 import torch
@@ -30,7 +32,7 @@ def _need_cuda():
 
 def _inputs(w):
     x = W.make_decode_inputs(w, "cpu")
-    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    return x, {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
 
 
 @pytest.mark.parametrize("name,over", [
@@ -39,7 +41,7 @@ def _inputs(w):
 ])
 def test_noalloc_matches_workspace_decode_on_two_calls(name, over):
     w = W.WORKLOADS[name].with_(**over)
-    xd = _inputs(w)
+    x, xd = _inputs(w)
     prob = bsa.problem_for(w, seq_lens=xd["seq_lens"], head_w=xd["head_w"])
     assert bsa.bsa_workspace_size(prob, bsa.OP_DECODE) <= bsa.NOALLOC_SCRATCH_BYTES
 
@@ -65,6 +67,12 @@ def test_noalloc_matches_workspace_decode_on_two_calls(name, over):
                                        step.lse.double().cpu().numpy())
         parity.check_attention(errs, f"no-alloc call {call}")
         assert parity.bf16_is_rne_of_f32(o.cpu(), o32.cpu())
+        # and against the fp64 oracle, row by row
+        out = SimpleNamespace(scores=step.scores, kept=step.kept, kept_count=step.kept_count,
+                              o=o, o_f32=o32, lse=lse)
+        rows = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+        s = parity.compare_decode_rows(w, x, out, rows)
+        assert s["rows"] == len(rows)
 
 
 def test_noalloc_rejects_problems_beyond_the_scratch_size():
