@@ -23,11 +23,15 @@
 //    per block, then the stage is released through its "empty" mbarrier.
 //  * 4-bit index keys (SpotAttention, Methodology §4; format in include/bsa.h):
 //    the same kernel streams 576-byte block records (9 B per token), with four
-//    CTAs per SM since the unpacking makes it latency- rather than HBM-bound. A lane turns its token's four 4-bit codes into
-//    bf16 with two byte-permute table lookups plus the sign bits (every code value
-//    is exact in bf16), runs the same MMA on the unscaled codes, and multiplies
-//    the token's ReLU head sum by its E4M3 scale (ReLU is positively homogeneous,
-//    and the scales are > 0); the cache scale g multiplies the block score.
+//    CTAs per SM. FP4 codes are E2M1 values (sign bit 3, exponent and mantissa in
+//    bits 0-2), so one hardware conversion turns a byte of two codes into an f16
+//    pair, exactly; the MMA then runs on f16 operands, with the index query
+//    converted to f16 once per row (exact for |q| in [2^-14, 65504]; a larger one
+//    is reported as BSA_DEV_FP16_RANGE). INT4 codes are turned into bf16 with two
+//    byte-permute table lookups plus the sign bits. Either way the MMA runs on the
+//    unscaled codes and the token's ReLU head sum is multiplied by its E4M3 scale
+//    (ReLU is positively homogeneous, and the scales are > 0); the cache scale g
+//    multiplies the block score.
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
 
@@ -93,6 +97,23 @@ BSA_DEVFN uint2 dequant4(uint32_t c16) {
   const uint32_t w0 = __byte_perm(lo, hi, 0x5140u) | (s0 & 0x80008000u);
   const uint32_t w1 = __byte_perm(lo, hi, 0x7362u) | (s1 & 0x80008000u);
   return make_uint2(w0, w1);
+}
+
+// Two FP4 (E2M1) codes in the low byte of x -> f16x2, the low nibble in the low half;
+// every E2M1 value is exact in f16.
+BSA_DEVFN uint32_t e2m1x2_to_f16x2(uint32_t x) {
+  uint32_t d;
+  asm("{\n .reg .b8 t;\n mov.b32 {t, _, _, _}, %1;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}"
+      : "=r"(d) : "r"(x));
+  return d;
+}
+
+// bf16x2 -> f16x2 (exact for magnitudes in [2^-14, 65504]); sets `big` when a value
+// is beyond the f16 range.
+BSA_DEVFN uint32_t bf16x2_to_f16x2(uint32_t x, bool& big) {
+  const float2 f = unpack_bf16(x);
+  big = big || fabsf(f.x) > 65504.f || fabsf(f.y) > 65504.f;
+  return pack_f16(f.x, f.y);
 }
 
 BSA_DEVFN int clamp_len(const ScoreDecodeArgs& a, int b) {
@@ -270,6 +291,12 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
               ((static_cast<int64_t>(b) * a.Hq + g * a.G + hl) * kR + 4 * tig) * 2);
           bq[nt][0] = v.x;
           bq[nt][1] = v.y;
+          if constexpr (KF == 1) {   // f16 MMA operands for FP4 keys
+            bool big = false;
+            bq[nt][0] = bf16x2_to_f16x2(v.x, big);
+            bq[nt][1] = bf16x2_to_f16x2(v.y, big);
+            if (big && tig == 0 && warp == 0) report(a.status, BSA_DEV_FP16_RANGE);
+          }
         }
         const int h0 = nt * 8 + 2 * tig, h1 = h0 + 1;
         // half weights: (w/2) * (c + |c|) = w * ReLU(c) exactly (c + |c| is 2c or +0)
@@ -298,6 +325,11 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
           if constexpr (KF == 0) {
             x0 = *reinterpret_cast<const uint2*>(blk + r0 * 32 + tig * 8);
             x1 = *reinterpret_cast<const uint2*>(blk + r1 * 32 + tig * 8);
+          } else if constexpr (KF == 1) {
+            const uint32_t c0 = *reinterpret_cast<const uint16_t*>(blk + r0 * 8 + tig * 2);
+            const uint32_t c1 = *reinterpret_cast<const uint16_t*>(blk + r1 * 8 + tig * 2);
+            x0 = make_uint2(e2m1x2_to_f16x2(c0), e2m1x2_to_f16x2(c0 >> 8));
+            x1 = make_uint2(e2m1x2_to_f16x2(c1), e2m1x2_to_f16x2(c1 >> 8));
           } else {
             x0 = dequant4<KF>(*reinterpret_cast<const uint16_t*>(blk + r0 * 8 + tig * 2));
             x1 = dequant4<KF>(*reinterpret_cast<const uint16_t*>(blk + r1 * 8 + tig * 2));
@@ -307,7 +339,8 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             float c[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_bf16(c, af, bq[nt][0], bq[nt][1]);
+            if constexpr (KF == 1) mma_f16(c, af, bq[nt][0], bq[nt][1]);
+            else mma_bf16(c, af, bq[nt][0], bq[nt][1]);
             // ReLU on the FMA pipe (the ALU pipe is the busier one)
             vr0 = fmaf(w0[nt], c[0] + fabsf(c[0]), vr0);
             vr0 = fmaf(w1[nt], c[1] + fabsf(c[1]), vr0);

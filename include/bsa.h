@@ -59,7 +59,8 @@ typedef enum {
 #define BSA_DEV_BAD_KEPT 0x2   /* kept block id outside [0, nb): skipped */
 #define BSA_DEV_NONFINITE 0x4  /* a block score was +-inf or NaN */
 #define BSA_DEV_TIMEOUT 0x8    /* a bounded wait inside a kernel gave up; outputs invalid */
-#define BSA_DEV_FP16_RANGE 0x10 /* prefill: a V value outside the fp16 range */
+#define BSA_DEV_FP16_RANGE 0x10 /* a value outside the fp16 range: a prefill V value, or an
+                                   index query scored against an FP4 index-key cache */
 
 typedef enum { BSA_PHASE_DECODE = 0, BSA_PHASE_PREFILL = 1 } bsa_phase_t;
 
