@@ -23,12 +23,13 @@ BSA_OK, BSA_ERR_INVALID_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_WORKSPACE, BSA_ERR_CUD
 BSA_DEV_BAD_PAGE, BSA_DEV_BAD_KEPT, BSA_DEV_NONFINITE, BSA_DEV_TIMEOUT, BSA_DEV_FP16_RANGE = (
     0x1, 0x2, 0x4, 0x8, 0x10)
 PHASE_DECODE, PHASE_PREFILL = 0, 1
-OP_SCORE, OP_SELECT, OP_DECODE, OP_PREFILL = 0, 1, 2, 3
+OP_SCORE, OP_SELECT, OP_DECODE, OP_PREFILL, OP_PBS_PERMUTE = 0, 1, 2, 3, 4
 BLOCK = 64
 
 EXPORTED = ["bsa_max_kept", "bsa_workspace_size", "bsa_score_blocks", "bsa_select_top_p",
             "bsa_decode", "bsa_prefill", "bsa_status_string", "bsa_last_cuda_error",
-            "bsa_decode_noalloc", "bsa_quantize_index_keys", "bsa_score_blocks_q"]
+            "bsa_decode_noalloc", "bsa_quantize_index_keys", "bsa_score_blocks_q",
+            "bsa_pbs_permute"]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 IDX_FP4, IDX_INT4 = 1, 2
 QIDX_RECORD_BYTES = 576
@@ -61,7 +62,8 @@ class CProblem(ctypes.Structure):
                 ("k_max", ctypes.c_int32), ("k_min", ctypes.c_int32), ("p", ctypes.c_float),
                 ("idx_scale", ctypes.c_float), ("attn_scale", ctypes.c_float),
                 ("head_w", ctypes.c_void_p), ("head_p", ctypes.c_void_p),
-                ("idx_heads", ctypes.c_int32)]
+                ("idx_heads", ctypes.c_int32), ("segment", ctypes.c_int32),
+                ("key_pos", ctypes.c_void_p)]
 
 
 _lib = None
@@ -95,6 +97,8 @@ def load_library(path: str = LIB_PATH):
     lib.bsa_quantize_index_keys.restype = ctypes.c_int
     lib.bsa_score_blocks_q.argtypes = [P, vp, CQCache, vp, vp, vp]
     lib.bsa_score_blocks_q.restype = ctypes.c_int
+    lib.bsa_pbs_permute.argtypes = [P, vp, CCache, CCache, CCache, vp, vp, vp, vp, vp, sz, vp, vp]
+    lib.bsa_pbs_permute.restype = ctypes.c_int
     lib.bsa_status_string.argtypes = [ctypes.c_int]
     lib.bsa_status_string.restype = ctypes.c_char_p
     lib.bsa_last_cuda_error.argtypes = []
@@ -144,6 +148,8 @@ class Problem:
     head_w: Optional[torch.Tensor] = None     # device float32 [Hq]
     head_p: Optional[torch.Tensor] = None     # device float32 [Hkv]: per-kv-head p (<= 0: local head)
     idx_heads: int = 0                        # 0: an index head per query head; 1: one per kv group
+    segment: int = 0                          # prefill: PBS segment length in tokens (0: none)
+    key_pos: Optional[torch.Tensor] = None    # prefill with segment: device int32 [B, Hkv, T]
 
     @property
     def G(self):
@@ -157,7 +163,8 @@ class Problem:
         return CProblem(self.phase, self.B, self.Hq, self.Hkv, self.d, self.r, self.block, self.T,
                         _ptr(self.seq_lens), self.n_sink, self.n_local, self.k_max, self.k_min,
                         float(self.p), float(self.idx_scale), float(self.attn_scale),
-                        _ptr(self.head_w), _ptr(self.head_p), int(self.idx_heads))
+                        _ptr(self.head_w), _ptr(self.head_p), int(self.idx_heads),
+                        int(self.segment), _ptr(self.key_pos))
 
 
 @dataclass
@@ -297,6 +304,16 @@ def bsa_decode_noalloc(prob: Problem, q, k: Cache, v: Cache, kept, kept_count, o
            "bsa_decode_noalloc")
 
 
+def bsa_pbs_permute(prob: Problem, q, k: Cache, v: Cache, k_idx: Cache, k_perm, v_perm,
+                    kidx_perm, key_pos, workspace, dev_status=None, stream=None):
+    _check(load_library().bsa_pbs_permute(ctypes.byref(prob.c()), _ptr(q), k.c(), v.c(),
+                                          k_idx.c(), _ptr(k_perm), _ptr(v_perm),
+                                          _ptr(kidx_perm), _ptr(key_pos), _ptr(workspace),
+                                          0 if workspace is None else workspace.numel(),
+                                          _ptr(dev_status), _stream(stream)),
+           "bsa_pbs_permute")
+
+
 def bsa_status_string(status: int) -> str:
     return load_library().bsa_status_string(status).decode()
 
@@ -367,6 +384,37 @@ class Prefill:
     def run(self, q, q_idx, k_idx: Cache, k: Cache, v: Cache, stream=None):
         self.select(q_idx, k_idx, stream)
         self.attend(q, k, v, stream)
+
+
+class PbsPrefill:
+    """Block-sparse prefill over a segment-permuted key order (PBS-Attn): permute the
+    keys inside segments of `prob.segment` tokens by importance, then score, select
+    and attend on the permuted caches. Buffers live in this object; ``run`` enqueues
+    the four entry points on the current stream."""
+
+    def __init__(self, prob: Problem, device="cuda", keep_f32=True):
+        assert prob.phase == PHASE_PREFILL and prob.segment > 0
+        dev = torch.device(device)
+        B, H, T, d = prob.B, prob.Hkv, prob.T, prob.d
+        self.k_perm = torch.empty(B, H, T, d, dtype=torch.bfloat16, device=dev)
+        self.v_perm = torch.empty(B, H, T, d, dtype=torch.bfloat16, device=dev)
+        self.kidx_perm = torch.empty(B, H, T, prob.r, dtype=torch.bfloat16, device=dev)
+        self.key_pos = torch.empty(B, H, T, dtype=torch.int32, device=dev)
+        prob.key_pos = self.key_pos
+        self.prob = prob
+        ws = bsa_workspace_size(prob, OP_PBS_PERMUTE)
+        self.pws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+        self.pf = Prefill(prob, device=device, keep_f32=keep_f32)
+        self.status = self.pf.status
+
+    def permute(self, q, k: Cache, v: Cache, k_idx: Cache, stream=None):
+        bsa_pbs_permute(self.prob, q, k, v, k_idx, self.k_perm, self.v_perm, self.kidx_perm,
+                        self.key_pos, self.pws, self.status, stream)
+
+    def run(self, q, q_idx, k_idx: Cache, k: Cache, v: Cache, stream=None):
+        self.permute(q, k, v, k_idx, stream)
+        self.pf.run(q, q_idx, contiguous_cache(self.kidx_perm), contiguous_cache(self.k_perm),
+                    contiguous_cache(self.v_perm), stream)
 
 
 def problem_for(w, seq_lens: Optional[torch.Tensor] = None,

@@ -94,8 +94,16 @@ bsa_status_t check_problem(const bsa_problem_t* p) {
   if (p->phase == BSA_PHASE_PREFILL && p->T <= 0) return BSA_ERR_INVALID_ARG;
   if (p->idx_heads != 0 && p->idx_heads != 1 && p->idx_heads != p->Hq / p->Hkv)
     return BSA_ERR_UNSUPPORTED;
+  if (p->segment != 0) {
+    if (p->phase != BSA_PHASE_PREFILL || p->segment < 0 || p->segment % 64 != 0)
+      return BSA_ERR_INVALID_ARG;
+    if (p->segment > 8192) return BSA_ERR_UNSUPPORTED;
+  }
   return BSA_OK;
 }
+
+// Blocks per segment of a permuted key order (1 when the keys keep their order).
+int seg_blocks_of(const bsa_problem_t* p) { return p->segment > 0 ? p->segment / 64 : 1; }
 
 // Index heads per kv group: one per query head (the default) or one per group
 // (SparDA, Main innovations §2: a compact indexer with one head per GQA group).
@@ -181,6 +189,21 @@ bsa::CacheView qview(const bsa_qcache_t& c) {
   return v;
 }
 
+// Workspace of bsa_pbs_permute: per-chunk row statistics, row log-sum-exps, importance.
+struct PbsWorkspace {
+  size_t ml, lse2, imp, total;
+};
+PbsWorkspace pbs_workspace(const bsa_problem_t* p) {
+  const size_t bh = static_cast<size_t>(p->B) * p->Hkv;
+  const size_t rows = bh * (p->Hq / p->Hkv) * 64;
+  PbsWorkspace w;
+  w.ml = 0;
+  w.lse2 = align256(rows * bsa::pbs_chunks(p->T) * 2 * sizeof(float));
+  w.imp = w.lse2 + align256(rows * sizeof(float));
+  w.total = w.imp + align256(bh * static_cast<size_t>(p->T) * sizeof(float));
+  return w;
+}
+
 }  // namespace
 
 namespace bsa {
@@ -192,7 +215,8 @@ extern "C" {
 int32_t bsa_max_kept(const bsa_problem_t* p) {
   if (p == nullptr) return 0;
   const int32_t base = p->n_sink + p->n_local + p->k_max;
-  return p->phase == BSA_PHASE_PREFILL ? base + 1 : base;
+  if (p->phase != BSA_PHASE_PREFILL) return base;
+  return base + (p->segment > 0 ? p->segment / 64 : 1);
 }
 
 bsa_status_t bsa_workspace_size(const bsa_problem_t* p, int32_t op, size_t* bytes) {
@@ -214,6 +238,11 @@ bsa_status_t bsa_workspace_size(const bsa_problem_t* p, int32_t op, size_t* byte
       if (p->phase != BSA_PHASE_PREFILL) return BSA_ERR_INVALID_ARG;
       const int64_t Tpad = static_cast<int64_t>(nblocks(p->T)) * 64;
       *bytes = align256(static_cast<size_t>(p->B) * p->Hkv * Tpad * p->d * 2) + 256;
+      return BSA_OK;
+    }
+    case BSA_OP_PBS_PERMUTE: {
+      if (p->phase != BSA_PHASE_PREFILL || p->segment <= 0) return BSA_ERR_INVALID_ARG;
+      *bytes = pbs_workspace(p).total;
       return BSA_OK;
     }
     default:
@@ -351,6 +380,7 @@ bsa_status_t bsa_select_top_p(const bsa_problem_t* p, const float* block_scores,
   a.k_min = p->k_min;
   a.p = p->p;
   a.head_p = p->head_p;
+  a.seg_blocks = seg_blocks_of(p);
   cudaError_t e = bsa::launch_select(a, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e);
 }
@@ -413,6 +443,7 @@ bsa_status_t bsa_prefill(const bsa_problem_t* p, const void* q, bsa_cache_t k, b
   if (q == nullptr || kept == nullptr || kept_count == nullptr || o == nullptr || lse == nullptr)
     return BSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(o) || (o_f32 && !aligned16(o_f32))) return BSA_ERR_INVALID_ARG;
+  if (p->segment > 0 && p->key_pos == nullptr) return BSA_ERR_INVALID_ARG;
   if ((st = check_cache(k, p, p->d, true)) != BSA_OK) return st;
   if ((st = check_cache(v, p, p->d, false)) != BSA_OK) return st;
   const int nqb = nblocks(p->T);
@@ -449,11 +480,62 @@ bsa_status_t bsa_prefill(const bsa_problem_t* p, const void* q, bsa_cache_t k, b
   a.Tpad = static_cast<int>(Tpad);
   a.max_kept = bsa_max_kept(p);
   a.scale_log2 = attn_scale_of(p) * 1.4426950408889634f;
+  a.seg_blocks = seg_blocks_of(p);
+  a.key_pos = p->segment > 0 ? p->key_pos : nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = bsa::launch_v_to_f16(a, s);
   if (e != cudaSuccess) return cuda_fail(e);
   int* unit_counter = reinterpret_cast<int*>(static_cast<char*>(workspace) + v16_bytes);
   e = bsa::launch_prefill_tc(a, tq, tk, tv, unit_counter, num_sms_current(), s);
+  return e == cudaSuccess ? BSA_OK : cuda_fail(e);
+}
+
+bsa_status_t bsa_pbs_permute(const bsa_problem_t* p, const void* q, bsa_cache_t k, bsa_cache_t v,
+                             bsa_cache_t k_idx, void* k_perm, void* v_perm, void* kidx_perm,
+                             int32_t* key_pos, void* workspace, size_t workspace_bytes,
+                             int32_t* dev_status, void* stream) {
+  bsa_status_t st = check_problem(p);
+  if (st != BSA_OK) return st;
+  if (p->phase != BSA_PHASE_PREFILL || p->segment <= 0) return BSA_ERR_INVALID_ARG;
+  if (q == nullptr || k_perm == nullptr || v_perm == nullptr || kidx_perm == nullptr ||
+      key_pos == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_perm) || !aligned16(v_perm) || !aligned16(kidx_perm) ||
+      !aligned16(key_pos))
+    return BSA_ERR_INVALID_ARG;
+  if ((st = check_cache(k, p, p->d, false)) != BSA_OK) return st;
+  if ((st = check_cache(v, p, p->d, false)) != BSA_OK) return st;
+  if ((st = check_cache(k_idx, p, p->r, false)) != BSA_OK) return st;
+  const PbsWorkspace ws = pbs_workspace(p);
+  if (workspace == nullptr || workspace_bytes < ws.total ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return BSA_ERR_WORKSPACE;
+  bsa::PbsArgs a{};
+  a.q = q;
+  a.k = view(k);
+  a.v = view(v);
+  a.kidx = view(k_idx);
+  a.k_perm = k_perm;
+  a.v_perm = v_perm;
+  a.kidx_perm = kidx_perm;
+  a.key_pos = key_pos;
+  char* w = static_cast<char*>(workspace);
+  a.ml = reinterpret_cast<float*>(w + ws.ml);
+  a.lse2 = reinterpret_cast<float*>(w + ws.lse2);
+  a.imp = reinterpret_cast<float*>(w + ws.imp);
+  a.status = dev_status;
+  a.B = p->B;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = p->Hq / p->Hkv;
+  a.d = p->d;
+  a.T = p->T;
+  a.nqb = nblocks(p->T);
+  a.nchunk = bsa::pbs_chunks(p->T);
+  a.segment = p->segment;
+  a.scale_log2 = attn_scale_of(p) * 1.4426950408889634f;
+  const cudaError_t e =
+      bsa::launch_pbs_permute(a, num_sms_current(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e);
 }
 

@@ -65,6 +65,7 @@ struct SelectArgs {
   const int32_t* seq_lens;
   int32_t* status;
   int phase, B, Hkv, T, nb_max, nqb, max_kept;
+  int seg_blocks;             // prefill: blocks per segment (1: the diagonal block alone)
   int n_sink, n_local, k_max, k_min;
   float p;
   const float* head_p;        // [Hkv] or null: per-head p
@@ -98,6 +99,24 @@ struct PrefillArgs {
   int32_t* status;
   int B, Hq, Hkv, G, d, T, nqb, Tpad, max_kept;
   float scale_log2;
+  int seg_blocks;             // blocks per segment of a permuted key order (1: none)
+  const int32_t* key_pos;     // [B*Hkv, T] original key positions of a permuted order, or null
+};
+
+// Segment permutation of the keys (PBS-Attn): importance, sort, gather.
+struct PbsArgs {
+  const void* q;              // [B, Hq, T, d] bf16
+  CacheView k, v, kidx;       // widths d, d, 16
+  void* k_perm;               // [B*Hkv, T, d] bf16
+  void* v_perm;               // [B*Hkv, T, d] bf16
+  void* kidx_perm;            // [B*Hkv, T, 16] bf16
+  int32_t* key_pos;           // [B*Hkv, T]
+  float* ml;                  // [B*Hkv, G*64, nchunk, 2] per-chunk (max, sum), log2 units
+  float* lse2;                // [B*Hkv, G*64] log-sum-exp of each last-block row, log2 units
+  float* imp;                 // [B*Hkv, T] importance
+  int32_t* status;
+  int B, Hq, Hkv, G, d, T, nqb, nchunk, segment;
+  float scale_log2;
 };
 
 // Launch with programmatic stream serialization: the kernel's CTAs may start while
@@ -130,6 +149,10 @@ cudaError_t launch_v_to_f16(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                               const CUtensorMap& tv16, int* unit_counter, int num_sms,
                               cudaStream_t s);
+
+cudaError_t launch_pbs_permute(const PbsArgs& a, int num_sms, cudaStream_t s);
+// Key chunks (CTAs per (b, g)) of the importance passes.
+int pbs_chunks(int T);
 
 // Blocks per work item of the decode scorer (items are (row, chunk) pairs).
 int score_decode_chunk_blocks();

@@ -114,11 +114,18 @@ BSA_DEVFN UnitInfo unit_of(const PrefillArgs& a, int u) {
   return U;
 }
 
+// First block of query block i's segment, and the end of the segment (with seg_blocks
+// = 1: i and i + 1).
+BSA_DEVFN int seg_begin(const PrefillArgs& a, int i) { return (i / a.seg_blocks) * a.seg_blocks; }
+BSA_DEVFN int seg_end(const PrefillArgs& a, int i) {
+  return min(seg_begin(a, i) + a.seg_blocks, a.nqb);
+}
+
 // Element offset of the first token of block `blk` in cache `c`, or -1 when the block
 // is not a valid kept block of query block i (out of range, bad page, past the extent).
 BSA_DEVFN int64_t block_off(const CacheView& c, const PrefillArgs& a, int b, int g, int blk,
                             int i) {
-  if (blk < 0 || blk > i) return -1;
+  if (blk < 0 || blk >= seg_end(a, i)) return -1;
   int64_t phys = blk;
   if (c.page_table != nullptr) {
     phys = c.page_table[static_cast<int64_t>(b) * c.pt_stride + blk];
@@ -182,9 +189,12 @@ BSA_DEVFN float2 exp2_poly(float2 x) {
 
 
 // Mask mode of a kept block: 0 visible, 1 the causal diagonal, 2 failed validation
-// (the loader then loads the diagonal block in its place).
+// (the loader then loads the diagonal block in its place), 3 a block of the query's
+// own segment of a permuted key order (a key is visible when its original position,
+// key_pos, is at most the query's; PBS-Attn, Methodology §2).
 BSA_DEVFN int mode_of(const PrefillArgs& a, const UnitInfo& U, int blk) {
   if (block_off(a.k, a, U.b, U.g, blk, U.i) < 0) return 2;
+  if (a.key_pos != nullptr) return blk >= seg_begin(a, U.i) ? 3 : 0;
   return blk == U.i ? 1 : 0;
 }
 
@@ -474,6 +484,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int blk = __shfl_sync(0xffffffffu, blk_v, jj & 31);
         const int mode = __shfl_sync(0xffffffffu, mode_v, jj & 31);
         const int buf = kc & 1;
+        // original positions of this thread's 16 keys (columns 8k + 2 t0, +1) of a block
+        // of the own segment; positions past T do not exist
+        int2 kp[8];
+        if (mode == 3) {
+          const int32_t* kpos = a.key_pos + (static_cast<int64_t>(U.b) * a.Hkv + U.g) * a.T;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int p = blk * kBlock + k * 8 + 2 * t0;
+            kp[k].x = p < a.T ? kpos[p] : 0x7fffffff;
+            kp[k].y = p + 1 < a.T ? kpos[p + 1] : 0x7fffffff;
+          }
+        }
         if (!warp_wait(&bars->s_full[t], kc & 1)) { ok = false; break; }
         tc::fence_after_sync();
         uint32_t sr[32];
@@ -483,8 +505,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_free[t]);
-        // masks: the causal diagonal block and blocks that failed validation
-        if (mode != 0) {
+        // masks: the causal diagonal block, blocks that failed validation, and the keys
+        // of the own segment that come after the query
+        if (mode == 3) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            if (kp[k].x > tqa) sr[4 * k] = 0xff800000u;
+            if (kp[k].y > tqa) sr[4 * k + 1] = 0xff800000u;
+            if (kp[k].x > tqb) sr[4 * k + 2] = 0xff800000u;
+            if (kp[k].y > tqb) sr[4 * k + 3] = 0xff800000u;
+          }
+        } else if (mode != 0) {
           const int dblk = mode == 2 ? 0 : blk;
           const int lima = mode == 2 ? -1 : tqa - dblk * kBlock;
           const int limb = mode == 2 ? -1 : tqb - dblk * kBlock;

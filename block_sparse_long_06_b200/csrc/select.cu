@@ -172,10 +172,14 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_
     c1 = max(c0, nbr - a.n_local);
     S = a.scores + static_cast<int64_t>(row) * a.nb_max;
   } else {
+    // the query block's segment [b0, b1) (its diagonal block when seg_blocks = 1) is
+    // kept; candidates are the earlier blocks outside the sinks and the n_local blocks
+    // before the segment (PBS-Attn, Methodology §2 for permuted segments)
     const int i = row % a.nqb;
-    nbr = i + 1;
-    c0 = min(a.n_sink, i);
-    c1 = max(c0, i - a.n_local);
+    const int b0 = (i / a.seg_blocks) * a.seg_blocks;
+    nbr = min(b0 + a.seg_blocks, a.nqb);
+    c0 = min(a.n_sink, b0);
+    c1 = max(c0, b0 - a.n_local);
     S = a.scores + static_cast<int64_t>(row) * a.nqb;
   }
   kept = a.kept + static_cast<int64_t>(row) * a.max_kept;

@@ -64,7 +64,8 @@ typedef enum {
 
 typedef enum { BSA_PHASE_DECODE = 0, BSA_PHASE_PREFILL = 1 } bsa_phase_t;
 
-typedef enum { BSA_OP_SCORE = 0, BSA_OP_SELECT = 1, BSA_OP_DECODE = 2, BSA_OP_PREFILL = 3 } bsa_op_t;
+typedef enum { BSA_OP_SCORE = 0, BSA_OP_SELECT = 1, BSA_OP_DECODE = 2, BSA_OP_PREFILL = 3,
+               BSA_OP_PBS_PERMUTE = 4 } bsa_op_t;
 
 /* Addressing of one bf16 cache tensor (K, V or index keys), contiguous or paged.
  * Token t of sequence b, kv head g starts at element
@@ -112,10 +113,20 @@ typedef struct {
                                has Hq rows and head_w Hq entries), 1 = one per group (SparDA,
                                Main innovations §2: a compact indexer; q_idx has Hkv rows,
                                head_w Hkv entries or NULL = 1). Other values: unsupported. */
+  int32_t segment;          /* prefill only: 0, or the segment length (tokens, a multiple of
+                               64, at most 8192) of a key order permuted inside segments by
+                               bsa_pbs_permute (PBS-Attn, Methodology §2-§4). Selection then
+                               keeps the query block's whole segment (instead of its diagonal
+                               block), the sinks and the n_local blocks before the segment,
+                               and chooses among the blocks of earlier segments. */
+  const int32_t* key_pos;   /* prefill with segment > 0: device [B, Hkv, T] original position
+                               of the key at each permuted position (bsa_pbs_permute's output);
+                               bsa_prefill masks the keys of the query's own segment by it */
 } bsa_problem_t;
 
 /* Length of one kept list: decode n_sink + n_local + k_max; prefill
- * 1 + n_sink + n_local + k_max. Unused slots of a list hold -1. */
+ * 1 + n_sink + n_local + k_max, or segment/64 + n_sink + n_local + k_max with a
+ * permuted key order (segment > 0). Unused slots of a list hold -1. */
 int32_t bsa_max_kept(const bsa_problem_t* prob);
 
 /* Workspace bytes `op` needs for `prob` (0 when none). Host only. */
@@ -162,6 +173,28 @@ bsa_status_t bsa_prefill(const bsa_problem_t* prob, const void* q, bsa_cache_t k
                          const int32_t* kept, const int32_t* kept_count, void* o, float* lse,
                          float* o_f32, void* workspace, size_t workspace_bytes,
                          int32_t* dev_status, void* stream);
+
+/* Segment permutation of the keys for block-sparse prefill (PBS-Attn, "Sparser
+ * Block-Sparse Attention via Token Permutation", Methodology §2-§3).
+ * For every (sequence b, kv head g) of a prefill problem with prob->segment = S > 0:
+ *   1. importance of key t = the mean, over the query rows of the last query block
+ *      (positions [64 * (nqb - 1), T)) of the group's query heads, of the causal
+ *      softmax probability that row gives t (scale attn_scale, keys t' <= the row's
+ *      position); computed in float32 in a fixed order;
+ *   2. inside each segment [s * S, min((s + 1) * S, T)) the keys are ordered by
+ *      importance descending, equal importance by lower position;
+ *   3. key_pos[b, g, p] = original position of the key at permuted position p, and
+ *      the permuted copies k_perm, v_perm [B, Hkv, T, d] and kidx_perm [B, Hkv, T, r]
+ *      (bf16, contiguous) hold row key_pos[b, g, p] of k, v and k_idx at row p.
+ * Queries are not permuted, so no output permutation has to be undone. The permuted
+ * caches then go to bsa_score_blocks, bsa_select_top_p and bsa_prefill with the same
+ * problem (segment and key_pos set). q is [B, Hq, T, d] bf16; k, v (width d) and
+ * k_idx (width r) are caches as elsewhere. Workspace: bsa_workspace_size with
+ * BSA_OP_PBS_PERMUTE. Runs four kernels on `stream`. */
+bsa_status_t bsa_pbs_permute(const bsa_problem_t* prob, const void* q, bsa_cache_t k,
+                             bsa_cache_t v, bsa_cache_t k_idx, void* k_perm, void* v_perm,
+                             void* kidx_perm, int32_t* key_pos, void* workspace,
+                             size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /* ------------------------------------------------------------------------
  * 4-bit index-key cache (SpotAttention, Methodology §4: the selector's K cache

@@ -114,12 +114,22 @@ def select_pbs(S_i: np.ndarray, i: int, seg_blocks: int, nqb: int, n_sink: int, 
 # --------------------------------------------------------------------------
 # whole rows
 # --------------------------------------------------------------------------
+def last_block_importance(q_g, K_g, T, attn_scale):
+    """Importance of every key from the last query block's rows (positions
+    [64 * (nqb - 1), T)) of the group's heads."""
+    ql = np.arange((O.num_blocks(T) - 1) * BLOCK, T)
+    return key_importance(q_g[:, ql, :], ql, K_g[:T], attn_scale)
+
+
 def pbs_prefill_rows(q_g, q_idx_g, k_idx_g, K_g, V_g, T, seg, head_w, idx_scale, attn_scale,
-                     n_sink, n_local, p, k_max, k_min=0, rows=None, kept_override=None):
+                     n_sink, n_local, p, k_max, k_min=0, rows=None, kept_override=None,
+                     perm_override=None):
     """PBS prefill for query blocks ``rows`` of one (sequence, kv head).
 
     q_g [G,>=T,d], q_idx_g [G,>=T,r], k_idx_g [>=T,r], K_g/V_g [>=T,d] in natural
-    order; seg = segment length in tokens (a multiple of 64).
+    order; seg = segment length in tokens (a multiple of 64). ``perm_override``
+    replaces the permutation (used to re-run the steps after it on an order that a
+    comparison accepted as a tie).
     Returns (perm, {i: dict(S, sel, o, lse)}): S are the scores of the permuted
     blocks [0, b0), o [G, n_q, d] and lse [G, n_q] in natural query order.
     """
@@ -128,9 +138,10 @@ def pbs_prefill_rows(q_g, q_idx_g, k_idx_g, K_g, V_g, T, seg, head_w, idx_scale,
     seg_blocks = seg // BLOCK
     rows = list(range(nqb)) if rows is None else list(rows)
     # importance from the last query block, then the segmented permutation
-    ql = np.arange((nqb - 1) * BLOCK, T)
-    imp = key_importance(q_g[:, ql, :], ql, K_g[:T], attn_scale)
-    perm = segment_permutation(imp, seg)
+    if perm_override is None:
+        perm = segment_permutation(last_block_importance(q_g, K_g, T, attn_scale), seg)
+    else:
+        perm = np.asarray(perm_override, dtype=np.int64)
     kidx_p = k_idx_g[:T][perm]
     out = {}
     for i in rows:

@@ -251,3 +251,84 @@ def compare_prefill_rows(w, inputs, pf, b, g, rows, check_scores=True, kept_dev=
     G = w.G
     assert bf16_is_rne_of_f32(o[b, g * G:(g + 1) * G], o32[b, g * G:(g + 1) * G])
     return summary
+
+
+# ------------------------------------------------------------------ PBS prefill rows
+IMP_TIE_REL = 1e-4   # importances this close (relative) may be ordered either way
+
+
+def permutation_verdict(imp, perm_dev, seg):
+    """'exact' | 'tie' | 'mismatch: ...' for a device key order against the oracle's
+    importances: every segment must hold its own positions, in an order whose
+    importance never rises by more than IMP_TIE_REL (relative) from one key to the
+    next, and keys of equal importance ordered by position."""
+    perm_dev = np.asarray(perm_dev, dtype=np.int64)
+    T = len(imp)
+    exact = True
+    for s0 in range(0, T, seg):
+        s1 = min(s0 + seg, T)
+        block = perm_dev[s0:s1]
+        if sorted(block.tolist()) != list(range(s0, s1)):
+            return f"mismatch: segment {s0} is not a permutation of its positions"
+        v = imp[block]
+        rise = v[1:] - v[:-1]
+        tol = np.maximum(IMP_TIE_REL * np.maximum(np.abs(v[1:]), np.abs(v[:-1])), 1e-30)
+        if np.any(rise > tol):
+            return f"mismatch: importance rises in segment {s0}"
+        eq = (v[1:] == v[:-1])
+        if np.any(eq & (block[1:] < block[:-1])):
+            return f"mismatch: equal importance out of position order in segment {s0}"
+        order = np.lexsort((np.arange(s0, s1), -imp[s0:s1]))
+        exact = exact and np.array_equal(block, np.arange(s0, s1)[order])
+    return "exact" if exact else "tie"
+
+
+def compare_pbs_rows(w, inputs, pbs, b, g, rows, seg):
+    """Compare a finished PbsPrefill with the PBS oracle on query blocks ``rows`` of
+    (b, g): key order (tie rule on importance), block scores of the earlier
+    segments, kept sets (tie rule on mass), attention."""
+    from oracle import pbs_oracle as P
+    G, T = w.G, w.T
+    q_g = f64(inputs["q"][b, g * G:(g + 1) * G, :T])
+    _, qi_g, hw = index_heads(inputs, w, b, g, (slice(0, T),))
+    ki_g = f64(inputs["k_idx"][b, g, :T])
+    K_g = f64(inputs["K"][b, g, :T])
+    V_g = f64(inputs["V"][b, g, :T])
+    args = (q_g, qi_g, ki_g, K_g, V_g, T, seg, hw, 1.0 / math.sqrt(w.r), 1.0 / math.sqrt(w.d),
+            w.n_sink, w.n_local, w.p, w.k_max, w.k_min)
+    summary = {"rows": 0, "ties": 0, "perm": "exact", "max_abs": 0.0, "rel_l2": 0.0,
+               "lse_abs": 0.0, "score_rel": 0.0}
+    kp = pbs.key_pos[b, g].cpu().numpy().astype(np.int64)
+    imp = P.last_block_importance(q_g, K_g, T, 1.0 / math.sqrt(w.d))
+    verdict = permutation_verdict(imp, kp, seg)
+    assert not verdict.startswith("mismatch"), f"key order of {(b, g)}: {verdict}"
+    summary["perm"] = verdict
+    perm, refs = P.pbs_prefill_rows(*args, rows=rows, perm_override=kp)
+    kept = pbs.pf.kept.cpu()
+    cnt = pbs.pf.kept_count.cpu()
+    scores = pbs.pf.scores.cpu()
+    o32 = pbs.pf.o_f32.cpu()
+    lse = pbs.pf.lse.cpu()
+    override = {}
+    for i, ref in refs.items():
+        nS = len(ref["S"])
+        if nS:
+            S_dev = scores[b, g, i, :nS].double().numpy()
+            rel = np.max(np.abs(S_dev - ref["S"]) / np.maximum(1.0, np.abs(ref["S"])))
+            summary["score_rel"] = max(summary["score_rel"], float(rel))
+            assert rel <= SCORE_REL, f"PBS row {(b, g, i)}: score rel err {rel}"
+        c = int(cnt[b, g, i])
+        kd = kept[b, g, i, :c].tolist()
+        assert all(x == -1 for x in kept[b, g, i, c:].tolist()), "padding is not -1"
+        v = selection_verdict(ref["sel"], kd, w.p)
+        assert not v.startswith("mismatch"), f"PBS row {(b, g, i)}: {v}"
+        if v == "tie":
+            summary["ties"] += 1
+            override[i] = kd
+    if override:
+        _, more = P.pbs_prefill_rows(*args, rows=list(override), kept_override=override,
+                                     perm_override=kp)
+        refs.update(more)
+    for i, ref in refs.items():
+        _check_prefill_block(w, o32, lse, b, g, i, ref, summary)
+    return summary
