@@ -387,6 +387,25 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline and do_dec and args.index_cache == "bf16":
         cpu = cpu_baseline_decode(wd, xd, dstep, budget_s=args.cpu_budget)
 
+    # other configurations of the path, each timed on its own (every rank runs them)
+    extras = {}
+    if not args.no_extras:
+        if do_dec and args.index_cache == "bf16":
+            qc = bsa.contiguous_qcache(wd.B, wd.Hkv, wd.T, bsa.IDX_FP4, device=dev)
+            bsa.bsa_quantize_index_keys(dprob, k_idx_c, qc, dstep.status)
+            extras["decode_fp4"] = time_decode(wd, xd, dprob, dstep, qc, K_c, V_c, "fp4", dev,
+                                               world, args.extra_steps, peaks)
+            del qc
+            del xd, dstep, K_c, V_c, k_idx_c
+            torch.cuda.empty_cache()
+            for key, name in (("decode_c2", "decode_b8_h32_t32k_paged"),
+                              ("decode_c4", "decode_b1_h64_t1m")):
+                extras[key] = time_decode_workload(name, rank, dev, world, args.extra_steps, peaks)
+        if do_pf:
+            extras["prefill_pbs"] = time_pbs(wp, xp, dev, world, 256, max(3, args.extra_steps // 4),
+                                             peaks)
+
+
     clocks = clk.summary()
     config = {"workload": " + ".join(w.name for w, on in ((wd, do_dec), (wp, do_pf)) if on)}
     if do_dec:
@@ -428,11 +447,90 @@ def run_ours(args, world, rank, local):
     line["roofline"] = roof_dec if roof_dec is not None else roof_pf
     if roof_dec is not None and roof_pf is not None:
         line["roofline_prefill"] = roof_pf
+    line.update(extras)
     line.update({"e2e": e2e, "gpu_launches": launches, "clocks": clocks,
                  "total_ms_events": total_ms})
     if cpu is not None:
         line["cpu_baseline"] = cpu
     return line
+
+
+def time_decode(w, xd, prob, step, k_idx, K, V, index_cache, dev, world, steps, peaks):
+    """Device time of the decode step (score -> select -> attend) on resident inputs,
+    a 256 MB buffer written before every step (untimed); mean over `steps`, max over
+    ranks."""
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(3):
+        step.run(xd["q"], xd["q_idx"], k_idx, K, V)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        step.run(xd["q"], xd["q_idx"], k_idx, K, V)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    st = int(step.status.item())
+    ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in evs) / steps, world)
+    by = decode_bytes(w, step.kept_count, xd["seq_lens"], index_cache)
+    gbs = by["step"] / (ms / 1e3) / 1e9
+    return {"workload": w.name, "index_cache": index_cache, "ms": ms,
+            "tokens_per_s": world * w.B / (ms / 1e3), "hbm_gbs": gbs,
+            "hbm_frac": gbs / peaks["hbm_gbs"], "bytes_per_step": by["step"], "steps": steps,
+            "device_status": st}
+
+
+def time_decode_workload(name, rank, dev, world, steps, peaks):
+    w = W.WORKLOADS[name].with_(seed=rank)
+    xd = W.make_decode_inputs(w, dev)
+    prob = bsa.problem_for(w, seq_lens=xd["seq_lens"], head_w=xd["head_w"])
+    step = bsa.DecodeStep(prob, device=dev, keep_f32=False)
+    k_idx, K, V = bsa.caches_for(xd)
+    out = time_decode(w, xd, prob, step, k_idx, K, V, "bf16", dev, world, steps, peaks)
+    out["config"] = describe(w)
+    del xd, step, K, V, k_idx
+    torch.cuda.empty_cache()
+    return out
+
+
+def time_pbs(w, xp, dev, world, segment, steps, peaks):
+    """Prefill over segment-permuted keys (PBS-Attn): permutation, score + select on the
+    permuted index keys, attention; the kept-tile FLOP over the attention time."""
+    prob = bsa.problem_for(w, head_w=xp["head_w"])
+    prob.segment = segment
+    pbs = bsa.PbsPrefill(prob, device=dev, keep_f32=False)
+    kc, K, V = (bsa.contiguous_cache(xp["k_idx"]), bsa.contiguous_cache(xp["K"]),
+                bsa.contiguous_cache(xp["V"]))
+    kcp, Kp, Vp = (bsa.contiguous_cache(pbs.kidx_perm), bsa.contiguous_cache(pbs.k_perm),
+                   bsa.contiguous_cache(pbs.v_perm))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(2):
+        pbs.run(xp["q"], xp["q_idx"], kc, K, V)
+    evs = []
+    for _ in range(steps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.zero_()
+        e[0].record(stream)
+        pbs.permute(xp["q"], K, V, kc)
+        e[1].record(stream)
+        pbs.pf.select(xp["q_idx"], kcp)
+        e[2].record(stream)
+        pbs.pf.attend(xp["q"], Kp, Vp)
+        e[3].record(stream)
+        evs.append(e)
+    torch.cuda.synchronize()
+    mean = lambda a, b: max_over_ranks(sum(e[a].elapsed_time(e[b]) for e in evs) / steps, world)
+    perm_ms, sel_ms, att_ms = mean(0, 1), mean(1, 2), mean(2, 3)
+    flops, flops_exact = prefill_flops(w, pbs.pf.kept_count)
+    tf = flops / (att_ms / 1e3) / 1e12
+    out = {"segment": segment, "permute_ms": perm_ms, "select_ms": sel_ms, "attention_ms": att_ms,
+           "tflops": world * tf, "tensor_frac": tf / peaks["bf16_tflops"],
+           "kept_tile_flop": flops, "steps": steps, "device_status": int(pbs.status.item())}
+    del pbs
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, dprob, dstep, xd, k_idx_c, K_c, V_c, stream, world):
@@ -572,6 +670,10 @@ def main():
     ap.add_argument("--prefill-workload", default=PREFILL_WL, choices=sorted(
         k for k, v in W.WORKLOADS.items() if v.phase == "prefill"))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other configurations (4-bit index cache, 32K and 1M decode, "
+                         "permuted-key prefill)")
+    ap.add_argument("--extra-steps", type=int, default=20)
     ap.add_argument("--idx-heads", type=int, choices=[0, 1], default=0,
                     help="prefill index heads per kv group: 0 = one per query head (the "
                          "method as configured), 1 = one per group (compact indexer)")
