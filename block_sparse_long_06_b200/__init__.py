@@ -63,7 +63,9 @@ class CProblem(ctypes.Structure):
                 ("idx_scale", ctypes.c_float), ("attn_scale", ctypes.c_float),
                 ("head_w", ctypes.c_void_p), ("head_p", ctypes.c_void_p),
                 ("idx_heads", ctypes.c_int32), ("segment", ctypes.c_int32),
-                ("key_pos", ctypes.c_void_p)]
+                ("key_pos", ctypes.c_void_p), ("group_size", ctypes.c_int32),
+                ("k_groups", ctypes.c_int32), ("group_scores", ctypes.c_void_p),
+                ("kept_groups", ctypes.c_void_p)]
 
 
 _lib = None
@@ -150,6 +152,10 @@ class Problem:
     idx_heads: int = 0                        # 0: an index head per query head; 1: one per kv group
     segment: int = 0                          # prefill: PBS segment length in tokens (0: none)
     key_pos: Optional[torch.Tensor] = None    # prefill with segment: device int32 [B, Hkv, T]
+    group_size: int = 0                       # decode: two-level routing group (16/32/64; 0: off)
+    k_groups: int = 0                         # decode with group_size: kept groups per row
+    group_scores: Optional[torch.Tensor] = None   # device float32 [B, Hkv, nb * 64 / group_size]
+    kept_groups: Optional[torch.Tensor] = None    # device int32 [B, Hkv, max_kept] bitmasks
 
     @property
     def G(self):
@@ -164,7 +170,8 @@ class Problem:
                         _ptr(self.seq_lens), self.n_sink, self.n_local, self.k_max, self.k_min,
                         float(self.p), float(self.idx_scale), float(self.attn_scale),
                         _ptr(self.head_w), _ptr(self.head_p), int(self.idx_heads),
-                        int(self.segment), _ptr(self.key_pos))
+                        int(self.segment), _ptr(self.key_pos), int(self.group_size),
+                        int(self.k_groups), _ptr(self.group_scores), _ptr(self.kept_groups))
 
 
 @dataclass
@@ -337,6 +344,11 @@ class DecodeStep:
         self.lse = torch.empty(prob.B, prob.Hq, dtype=torch.float32, device=dev)
         self.o_f32 = (torch.empty(prob.B, prob.Hq, prob.d, dtype=torch.float32, device=dev)
                       if keep_f32 else None)
+        if prob.group_size > 0:   # two-level routing: group scores and kept-group masks
+            prob.group_scores = torch.empty(prob.B, prob.Hkv, prob.nb * BLOCK // prob.group_size,
+                                            dtype=torch.float32, device=dev)
+            prob.kept_groups = torch.empty(prob.B, prob.Hkv, mk, dtype=torch.int32, device=dev)
+            self.group_scores, self.kept_groups = prob.group_scores, prob.kept_groups
         ws = bsa_workspace_size(prob, OP_DECODE)
         self.workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)

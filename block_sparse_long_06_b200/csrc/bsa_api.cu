@@ -53,13 +53,15 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 2-D map over rows of `width` 16-bit elements, 64 x 64 boxes, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int width, bool fp16) {
+// 2-D map over rows of `width` 16-bit elements, 64-wide boxes of `box_rows` rows,
+// 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int width, bool fp16,
+              int box_rows = 64) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(width), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(width) * 2};
-  cuuint32_t box[2] = {64, 64};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    const_cast<void*>(base), dims, strides, box, estr,
@@ -98,6 +100,12 @@ bsa_status_t check_problem(const bsa_problem_t* p) {
     if (p->phase != BSA_PHASE_PREFILL || p->segment < 0 || p->segment % 64 != 0)
       return BSA_ERR_INVALID_ARG;
     if (p->segment > 8192) return BSA_ERR_UNSUPPORTED;
+  }
+  if (p->group_size != 0) {
+    if (p->phase != BSA_PHASE_DECODE || p->k_groups < 0) return BSA_ERR_INVALID_ARG;
+    if (p->group_size != 16 && p->group_size != 32 && p->group_size != 64)
+      return BSA_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(p->k_max) * (64 / p->group_size) > 8192) return BSA_ERR_UNSUPPORTED;
   }
   return BSA_OK;
 }
@@ -255,6 +263,7 @@ bsa_status_t bsa_score_blocks(const bsa_problem_t* p, const void* q_idx, bsa_cac
   bsa_status_t st = check_problem(p);
   if (st != BSA_OK) return st;
   if (q_idx == nullptr || block_scores == nullptr || !aligned16(q_idx)) return BSA_ERR_INVALID_ARG;
+  if (p->group_size > 0 && p->group_scores == nullptr) return BSA_ERR_INVALID_ARG;
   if ((st = check_cache(k_idx, p, p->r, false)) != BSA_OK) return st;
   const int num_sms = num_sms_current();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -279,6 +288,8 @@ bsa_status_t bsa_score_blocks(const bsa_problem_t* p, const void* q_idx, bsa_cac
     a.chunks_per_row = (a.nb_max + cb - 1) / cb;
     a.total_items = static_cast<int64_t>(p->B) * p->Hkv * a.chunks_per_row;
     a.idx_scale = idx_scale_of(p);
+    a.group_size = p->group_size;
+    a.group_scores = p->group_scores;
     e = bsa::launch_score_decode(a, num_sms, s);
   } else {
     bsa::ScorePrefillArgs a{};
@@ -329,6 +340,7 @@ bsa_status_t bsa_score_blocks_q(const bsa_problem_t* p, const void* q_idx, bsa_q
   if (st != BSA_OK) return st;
   if (p->phase != BSA_PHASE_DECODE) return BSA_ERR_UNSUPPORTED;
   if (q_idx == nullptr || block_scores == nullptr || !aligned16(q_idx)) return BSA_ERR_INVALID_ARG;
+  if (p->group_size > 0 && p->group_scores == nullptr) return BSA_ERR_INVALID_ARG;
   if ((st = check_qcache(k_idx, p)) != BSA_OK) return st;
   bsa::ScoreDecodeArgs a{};
   a.q_idx = q_idx;
@@ -351,6 +363,8 @@ bsa_status_t bsa_score_blocks_q(const bsa_problem_t* p, const void* q_idx, bsa_q
   a.idx_scale = idx_scale_of(p);
   a.kfmt = k_idx.format;
   a.gscale = k_idx.gscale;
+  a.group_size = p->group_size;
+  a.group_scores = p->group_scores;
   const cudaError_t e = bsa::launch_score_decode(a, num_sms_current(), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e);
 }
@@ -360,6 +374,8 @@ bsa_status_t bsa_select_top_p(const bsa_problem_t* p, const float* block_scores,
   bsa_status_t st = check_problem(p);
   if (st != BSA_OK) return st;
   if (block_scores == nullptr || kept == nullptr || kept_count == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (p->group_size > 0 && (p->group_scores == nullptr || p->kept_groups == nullptr))
     return BSA_ERR_INVALID_ARG;
   bsa::SelectArgs a{};
   a.scores = block_scores;
@@ -382,6 +398,27 @@ bsa_status_t bsa_select_top_p(const bsa_problem_t* p, const float* block_scores,
   a.head_p = p->head_p;
   a.seg_blocks = seg_blocks_of(p);
   cudaError_t e = bsa::launch_select(a, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess && p->group_size > 0) {
+    // level 2: the best token groups of the kept blocks
+    bsa::GroupSelectArgs ga{};
+    ga.group_scores = p->group_scores;
+    ga.kept = kept;
+    ga.kept_count = kept_count;
+    ga.seq_lens = p->seq_lens;
+    ga.kept_groups = p->kept_groups;
+    ga.status = dev_status;
+    ga.B = p->B;
+    ga.Hkv = p->Hkv;
+    ga.T = p->T;
+    ga.nb_max = nblocks(p->T);
+    ga.max_kept = a.max_kept;
+    ga.n_sink = p->n_sink;
+    ga.n_local = p->n_local;
+    ga.group_size = p->group_size;
+    ga.k_groups = p->k_groups;
+    ga.max_cand = p->k_max * (64 / p->group_size);
+    e = bsa::launch_select_groups(ga, static_cast<cudaStream_t>(stream));
+  }
   return e == cudaSuccess ? BSA_OK : cuda_fail(e);
 }
 
@@ -402,10 +439,19 @@ bsa_status_t bsa_decode(const bsa_problem_t* p, const void* q, bsa_cache_t k, bs
   const size_t need = align256(pl.part_o_bytes) + align256(pl.part_ml_bytes);
   if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return BSA_ERR_WORKSPACE;
-  CUtensorMap tk, tv;
+  if (p->group_size > 0 && p->kept_groups == nullptr) return BSA_ERR_INVALID_ARG;
+  CUtensorMap tk, tv, tk16, tv16;
   if (!make_map(&tk, k.base, k.extent / p->d, p->d, false) ||
       !make_map(&tv, v.base, v.extent / p->d, p->d, false))
     return cuda_fail(cudaErrorInvalidValue);
+  if (p->group_size > 0) {
+    if (!make_map(&tk16, k.base, k.extent / p->d, p->d, false, 16) ||
+        !make_map(&tv16, v.base, v.extent / p->d, p->d, false, 16))
+      return cuda_fail(cudaErrorInvalidValue);
+  } else {
+    tk16 = tk;   // not read: every kept block is copied whole
+    tv16 = tv;
+  }
   bsa::DecodeArgs a{};
   a.q = q;
   a.k = view(k);
@@ -429,7 +475,10 @@ bsa_status_t bsa_decode(const bsa_problem_t* p, const void* q, bsa_cache_t k, bs
   a.splits = pl.splits;
   a.split_len = pl.split_len;
   a.scale_log2 = attn_scale_of(p) * 1.4426950408889634f;
-  cudaError_t e = bsa::launch_decode(a, tk, tv, pl.units, num_sms, static_cast<cudaStream_t>(stream));
+  a.kept_groups = p->group_size > 0 ? p->kept_groups : nullptr;
+  a.group_size = p->group_size;
+  cudaError_t e = bsa::launch_decode(a, tk, tv, tk16, tv16, pl.units, num_sms,
+                                     static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e);
 }
 

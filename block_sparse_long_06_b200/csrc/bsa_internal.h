@@ -32,6 +32,8 @@ struct ScoreDecodeArgs {
   float idx_scale;
   int kfmt;                   // 0: bf16 keys; 1: FP4 / 2: INT4 records (kidx counts records)
   const float* gscale;        // 4-bit formats: the cache scale g (device)
+  int group_size;             // 0, or 16 / 32 / 64: also write group maxima
+  float* group_scores;        // [B*Hkv, nb_max * 64 / group_size]
 };
 
 // 4-bit index-key cache: 576-byte records of 64 tokens (codes, then scales).
@@ -71,6 +73,18 @@ struct SelectArgs {
   const float* head_p;        // [Hkv] or null: per-head p
 };
 
+// Level-2 routing of decode rows: the best groups of the dynamically kept blocks.
+struct GroupSelectArgs {
+  const float* group_scores;  // [B*Hkv, nb_max * gpb]
+  const int32_t* kept;        // [B*Hkv, max_kept]
+  const int32_t* kept_count;  // [B*Hkv]
+  const int32_t* seq_lens;
+  int32_t* kept_groups;       // [B*Hkv, max_kept] bitmasks
+  int32_t* status;
+  int B, Hkv, T, nb_max, max_kept, n_sink, n_local, group_size, k_groups;
+  int max_cand;               // k_max * 64 / group_size: candidate groups of a row, at most
+};
+
 struct DecodeArgs {
   const void* q;              // [B, Hq, d] bf16
   CacheView k, v;
@@ -82,6 +96,8 @@ struct DecodeArgs {
   float* o_f32;               // [B, Hq, d] or null
   float* part_o;              // [units, G, d]
   float* part_ml;             // [units, G, 2]
+  const int32_t* kept_groups; // [B*Hkv, max_kept] group bitmasks, or null (whole blocks)
+  int group_size;
   int32_t* status;
   int B, Hq, Hkv, G, d, T, max_kept, splits, split_len;
   float scale_log2;           // attn_scale * log2(e)
@@ -143,8 +159,11 @@ cudaError_t launch_score_decode(const ScoreDecodeArgs& a, int num_sms, cudaStrea
 cudaError_t launch_quantize_index(const QuantArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_score_prefill(const ScorePrefillArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
+cudaError_t launch_select_groups(const GroupSelectArgs& a, cudaStream_t s);
+// tk16 / tv16: the same caches with 16-row boxes (copies of partly kept blocks).
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                          int num_units, int num_sms, cudaStream_t s);
+                          const CUtensorMap& tk16, const CUtensorMap& tv16, int num_units,
+                          int num_sms, cudaStream_t s);
 cudaError_t launch_v_to_f16(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                               const CUtensorMap& tv16, int* unit_counter, int num_sms,

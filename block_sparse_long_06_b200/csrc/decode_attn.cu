@@ -19,6 +19,11 @@
 //  * at the end of a unit the four warps' (m, l, O) are merged in shared memory
 //    and written as one partial; the merge kernel combines the splits of a row
 //    with their log-sum-exp weights and writes o (bf16), o_f32 and lse.
+//  * two-level routing (HGA, Central mechanism §2): each kept entry carries a
+//    bitmask of its kept token groups. A block with every group kept is copied as
+//    above; otherwise only the 16-token quarters of its kept groups are copied
+//    (16-row boxes at the same swizzled offsets), and a consumer warp whose
+//    quarter was not copied skips the block.
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
 
@@ -83,7 +88,9 @@ BSA_DEVFN int64_t tile_row(const CacheView& c, int b, int g, int blk, int rows, 
 template <int D, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_attn_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
-                       const __grid_constant__ CUtensorMap tmv, const int num_units) {
+                       const __grid_constant__ CUtensorMap tmv,
+                       const __grid_constant__ CUtensorMap tmk16,
+                       const __grid_constant__ CUtensorMap tmv16, const int num_units) {
   using Cfg = DecodeCfg<D>;
   using Sm = DecodeSmem<D, NT>;
   constexpr int S = Cfg::kStages;
@@ -117,6 +124,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       prefetch_tensormap(&tmk);
       prefetch_tensormap(&tmv);
+      if (a.kept_groups != nullptr) {
+        prefetch_tensormap(&tmk16);
+        prefetch_tensormap(&tmv16);
+      }
     }
     uint32_t it = 0;
     bool ok_all = true;
@@ -129,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nb = (Tb + kBlock - 1) / kBlock;
       for (int base = e0; base < e1 && ok_all; base += 32) {
         const int e = base + lane;
-        int blk = -1;
+        int blk = -1, qm = 15;   // qm: 16-token quarters to copy and attend
         int64_t rk = -1, rv = -1;
         if (e < e1) {
           blk = a.kept[static_cast<int64_t>(row) * a.max_kept + e];
@@ -138,6 +149,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             rk = tile_row(a.k, b, g, blk, rows, D);
             rv = tile_row(a.v, b, g, blk, rows, D);
             if (rk < 0 || rv < 0) report(a.status, BSA_DEV_BAD_PAGE);
+            if (a.kept_groups != nullptr) {
+              const uint32_t gm = static_cast<uint32_t>(
+                  a.kept_groups[static_cast<int64_t>(row) * a.max_kept + e]);
+              qm = 0;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) qm |= static_cast<int>((gm >> (q * 16 / a.group_size)) & 1u) << q;
+              // a partly kept block: only its quarters that hold tokens
+              if (qm != 15) qm &= (1 << ((rows + 15) / 16)) - 1;
+            }
           } else {
             report(a.status, BSA_DEV_BAD_KEPT);
           }
@@ -147,22 +167,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int blk_q = __shfl_sync(0xffffffffu, blk, q);
           const int64_t rk_q = __shfl_sync(0xffffffffu, rk, q);
           const int64_t rv_q = __shfl_sync(0xffffffffu, rv, q);
+          const int qm_q = __shfl_sync(0xffffffffu, qm, q);
           if (lane == 0) {
             const int s = it % S;
             if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
               report(a.status, BSA_DEV_TIMEOUT);
               ok_all = false;
             } else {
-              const bool ok = rk_q >= 0 && rv_q >= 0;
-              sinfo[s] = ok ? blk_q : -1;
+              const bool ok = rk_q >= 0 && rv_q >= 0 && qm_q != 0;
+              sinfo[s] = ok ? (blk_q << 4) | qm_q : -1;
               unsigned char* st = ring + s * Cfg::kStageBytes;
-              if (ok) {
+              if (ok && qm_q == 15) {
                 mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
 #pragma unroll
                 for (int x = 0; x < Cfg::kBoxes; ++x) {
                   tma_load_2d(st + x * 8192, &tmk, x * 64, static_cast<int32_t>(rk_q), &full[s]);
                   tma_load_2d(st + Cfg::kTileBytes + x * 8192, &tmv, x * 64,
                               static_cast<int32_t>(rv_q), &full[s]);
+                }
+              } else if (ok) {
+                // kept quarters only: 16 rows x 64 dims per box, 2 KB apart in the tile
+                mbar_arrive_expect_tx(&full[s], __popc(qm_q) * Cfg::kStageBytes / 4);
+                for (int q4 = 0; q4 < 4; ++q4) {
+                  if (!((qm_q >> q4) & 1)) continue;
+#pragma unroll
+                  for (int x = 0; x < Cfg::kBoxes; ++x) {
+                    tma_load_2d(st + x * 8192 + q4 * 2048, &tmk16, x * 64,
+                                static_cast<int32_t>(rk_q + 16 * q4), &full[s]);
+                    tma_load_2d(st + Cfg::kTileBytes + x * 8192 + q4 * 2048, &tmv16, x * 64,
+                                static_cast<int32_t>(rv_q + 16 * q4), &full[s]);
+                  }
                 }
               } else {
                 mbar_arrive(&full[s]);
@@ -229,8 +263,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         alive = false;
         break;
       }
-      const int blk = sinfo[s];
-      if (blk >= 0) {
+      const int info = sinfo[s];
+      const int blk = info >> 4;   // -1 when nothing was copied
+      if (info >= 0 && ((info >> warp) & 1)) {
         const uint32_t kb = smem_u32(ring + s * Cfg::kStageBytes);
         const uint32_t vb = kb + Cfg::kTileBytes;
         const int valid = Tb - blk * kBlock - 16 * warp;  // tokens of this warp that exist
@@ -421,14 +456,15 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a) {
 
 template <int D, int NT>
 cudaError_t launch_dn(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                      int num_units, int num_sms, cudaStream_t s) {
+                      const CUtensorMap& tk16, const CUtensorMap& tv16, int num_units,
+                      int num_sms, cudaStream_t s) {
   const int smem = DecodeSmem<D, NT>::kTotal;
   auto kern = decode_attn_kernel<D, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = num_units < num_sms ? num_units : num_sms;
   if (grid > 0) {
-    e = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, a, tk, tv, num_units);
+    e = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, s, a, tk, tv, tk16, tv16, num_units);
     if (e != cudaSuccess) return e;
   }
   const int warps = a.B * a.Hq;
@@ -457,14 +493,15 @@ void decode_split_plan(int rows, int max_kept, int num_sms, int* splits, int* sp
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                          int num_units, int num_sms, cudaStream_t s) {
+                          const CUtensorMap& tk16, const CUtensorMap& tv16, int num_units,
+                          int num_sms, cudaStream_t s) {
   const int NT = a.G > 8 ? 2 : 1;
   if (a.d == 128) {
-    return NT == 1 ? launch_dn<128, 1>(a, tk, tv, num_units, num_sms, s)
-                   : launch_dn<128, 2>(a, tk, tv, num_units, num_sms, s);
+    return NT == 1 ? launch_dn<128, 1>(a, tk, tv, tk16, tv16, num_units, num_sms, s)
+                   : launch_dn<128, 2>(a, tk, tv, tk16, tv16, num_units, num_sms, s);
   }
-  return NT == 1 ? launch_dn<64, 1>(a, tk, tv, num_units, num_sms, s)
-                 : launch_dn<64, 2>(a, tk, tv, num_units, num_sms, s);
+  return NT == 1 ? launch_dn<64, 1>(a, tk, tv, tk16, tv16, num_units, num_sms, s)
+                 : launch_dn<64, 2>(a, tk, tv, tk16, tv16, num_units, num_sms, s);
 }
 
 }  // namespace bsa

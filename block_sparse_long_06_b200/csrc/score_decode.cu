@@ -32,6 +32,8 @@
 //    unscaled codes and the token's ReLU head sum is multiplied by its E4M3 scale
 //    (ReLU is positively homogeneous, and the scales are > 0); the cache scale g
 //    multiplies the block score.
+//  * with group_size > 0 (two-level routing) the same token scores also give the
+//    max of every group of 16, 32 or 64 tokens, written beside the block scores.
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
 
@@ -307,16 +309,18 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
     if (j < a.nb_max) {
       float* out = a.scores + static_cast<int64_t>(in.row) * a.nb_max + j;
       const int valid = in.Tb - j * kBlock;  // tokens of this block that exist
-      if (valid <= 0) {
-        if (lane == 0) *out = -INFINITY;
-      } else if (!(in.ok & (1u << warp))) {
+      const int gpb = a.group_size > 0 ? kBlock / a.group_size : 0;
+      float* gout = gpb ? a.group_scores + (static_cast<int64_t>(in.row) * a.nb_max + j) * gpb : nullptr;
+      if (valid <= 0 || !(in.ok & (1u << warp))) {
         if (lane == 0) {
           *out = -INFINITY;
-          report(a.status, BSA_DEV_BAD_PAGE);
+          if (valid > 0) report(a.status, BSA_DEV_BAD_PAGE);
         }
+        if (lane < gpb) gout[lane] = -INFINITY;
       } else {
         const unsigned char* blk = ring + s * kStageBytes + warp * kBlockBytes;
         float mx = 0.f;
+        float gm[4];   // this lane's token score of each 16-token group (-inf past the end)
         const bool odd = tig & 1;
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
@@ -356,6 +360,26 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
           const int tok = odd ? r1 : r0;
           if constexpr (KF != 0) keep *= scale_lut[blk[kBlock * 8 + tok] & 0x7Fu];   // token scale
           if (tok < valid) mx = fmaxf(mx, keep);
+          gm[mt] = tok < valid ? keep : -INFINITY;
+        }
+        if (gpb) {
+          // group maxima (HGA, Central mechanism §2: group summaries, here the max of
+          // the group's token scores): a transposing butterfly reduces the four
+          // 16-token groups in 6 shuffles; lane 8m ends with group m.
+          const bool h16 = lane & 16, h8 = lane & 8;
+          float k0 = h16 ? gm[2] : gm[0], k1 = h16 ? gm[3] : gm[1];
+          k0 = fmaxf(k0, __shfl_xor_sync(0xffffffffu, h16 ? gm[0] : gm[2], 16));
+          k1 = fmaxf(k1, __shfl_xor_sync(0xffffffffu, h16 ? gm[1] : gm[3], 16));
+          float gk = h8 ? k1 : k0;
+          gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8));
+          gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, 4));
+          gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, 2));
+          gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, 1));
+          if (gpb <= 2) gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, 8));    // 32-token groups
+          if (gpb == 1) gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, 16));   // one group
+          const int step = 32 / gpb;   // lane of group m: m * step
+          if ((lane & (step - 1)) == 0)
+            gout[lane / step] = gk == -INFINITY ? -INFINITY : a.idx_scale * (kscale * gk);
         }
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));

@@ -137,6 +137,70 @@ BSA_DEVFN T block_exscan(T v, T* scratch, T& total) {
   return base + inc - v;
 }
 
+// Radix select over keys[skew(0 .. n)) (4 passes x 8 bits, warp-aggregated shared-memory
+// histograms, integer counts only): returns the rem-th smallest key (1-based) and leaves
+// in `rem` how many keys equal to it are among the rem smallest (every smaller key is).
+template <int NT>
+BSA_DEVFN uint32_t radix_kth(const uint32_t* keys, int n, int& rem, uint32_t* hist,
+                             uint32_t* s_bucket_info) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t prefix = 0u, pmask = 0u;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int x = tid; x < kHistCopies * 256; x += NT) hist[x] = 0u;
+    __syncthreads();
+    uint32_t* h = hist + (warp % kHistCopies) * 256;
+    for (int t0 = 0; t0 < n; t0 += NT) {
+      const int t = t0 + tid;
+      uint32_t digit = 256u;
+      if (t < n) {
+        const uint32_t k = keys[skew(t)];
+        if ((k & pmask) == prefix) digit = (k >> shift) & 255u;
+      }
+      hist_add(h, digit, pass, lane);
+    }
+    __syncthreads();
+    for (int x = tid; x < 256; x += NT) {
+      uint32_t tot = 0;
+      for (int c = 0; c < kHistCopies; ++c) tot += hist[c * 256 + x];
+      hist[x] = tot;  // copy 0 now holds totals (other copies no longer needed)
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t part = 0;
+      for (int q = 0; q < 8; ++q) part += hist[lane * 8 + q];
+      uint32_t inc = part;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t nn = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += nn;
+      }
+      const uint32_t exc = inc - part;
+      const bool here = (exc < static_cast<uint32_t>(rem)) && (inc >= static_cast<uint32_t>(rem));
+      if (here) {
+        uint32_t c = exc;
+        int bsel = lane * 8;
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t hq = hist[lane * 8 + q];
+          if (c + hq >= static_cast<uint32_t>(rem)) {
+            bsel = lane * 8 + q;
+            break;
+          }
+          c += hq;
+        }
+        s_bucket_info[0] = static_cast<uint32_t>(bsel);
+        s_bucket_info[1] = c;  // count strictly below the bucket
+      }
+    }
+    __syncthreads();
+    prefix |= s_bucket_info[0] << shift;
+    pmask |= 255u << shift;
+    rem -= static_cast<int>(s_bucket_info[1]);
+    __syncthreads();
+  }
+  return prefix;
+}
+
 template <int NT>
 __global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_nc, int sort_n) {
   constexpr int NW = NT / 32;
@@ -209,61 +273,8 @@ __global__ void __launch_bounds__(NT) select_kernel(const SelectArgs a, int max_
   int kdyn = 0;
   if (kcap > 0 && kcap < nC) {
     // ---- 2. radix select of the kcap-th key ------------------------------------
-    uint32_t prefix = 0u, pmask = 0u;
     int rem = kcap;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int x = tid; x < kHistCopies * 256; x += NT) hist[x] = 0u;
-      __syncthreads();
-      uint32_t* h = hist + (warp % kHistCopies) * 256;
-      for (int t0 = 0; t0 < nC; t0 += NT) {
-        const int t = t0 + tid;
-        uint32_t digit = 256u;
-        if (t < nC) {
-          const uint32_t k = keys[skew(t)];
-          if ((k & pmask) == prefix) digit = (k >> shift) & 255u;
-        }
-        hist_add(h, digit, pass, lane);
-      }
-      __syncthreads();
-      for (int x = tid; x < 256; x += NT) {
-        uint32_t tot = 0;
-        for (int c = 0; c < kHistCopies; ++c) tot += hist[c * 256 + x];
-        hist[x] = tot;  // copy 0 now holds totals (other copies no longer needed)
-      }
-      __syncthreads();
-      if (warp == 0) {
-        uint32_t part = 0;
-        for (int q = 0; q < 8; ++q) part += hist[lane * 8 + q];
-        uint32_t inc = part;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
-          if (lane >= o) inc += n;
-        }
-        const uint32_t exc = inc - part;
-        const bool here = (exc < static_cast<uint32_t>(rem)) && (inc >= static_cast<uint32_t>(rem));
-        if (here) {
-          uint32_t c = exc;
-          int bsel = lane * 8;
-          for (int q = 0; q < 8; ++q) {
-            const uint32_t hq = hist[lane * 8 + q];
-            if (c + hq >= static_cast<uint32_t>(rem)) {
-              bsel = lane * 8 + q;
-              break;
-            }
-            c += hq;
-          }
-          s_bucket_info[0] = static_cast<uint32_t>(bsel);
-          s_bucket_info[1] = c;  // count strictly below the bucket
-        }
-      }
-      __syncthreads();
-      prefix |= s_bucket_info[0] << shift;
-      pmask |= 255u << shift;
-      rem -= static_cast<int>(s_bucket_info[1]);
-      __syncthreads();
-    }
+    const uint32_t prefix = radix_kth<NT>(keys, nC, rem, hist, s_bucket_info);
     // keys < prefix are in; among keys == prefix take the `rem` lowest ids
     int neq = 0;
     for (int t = seg0; t < seg1; ++t) neq += (keys[skew(t)] == prefix);
@@ -373,6 +384,102 @@ emit:
   const int count = c0 + tot + nlocal;
   for (int x = count + tid; x < a.max_kept; x += NT) kept[x] = -1;
   if (tid == 0) *kcount = count;
+}
+
+// Level-2 routing of a decode row (HGA, Central mechanism §2): the groups of
+// group_size tokens of the row's dynamically kept blocks are the candidates, in
+// ascending group id (the kept list is ascending); the k_groups of highest group
+// score are kept (ties to the lower group id: equal keys in enumeration order), by
+// the same radix select as the blocks. Sink and local entries keep every group. Out:
+// one bitmask per kept-list entry (bit k = group k of the block), 0 past the count.
+template <int NT>
+__global__ void __launch_bounds__(NT) select_groups_kernel(const GroupSelectArgs a) {
+  constexpr int NW = NT / 32;
+  extern __shared__ __align__(16) unsigned char smem[];
+  // layout: [block ids: max_kept i32][keys: skew(max_cand) u32][hist: copies*256 u32][flags]
+  int32_t* ids = reinterpret_cast<int32_t*>(smem);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(ids + a.max_kept);
+  uint32_t* hist = keys + skew(a.max_cand) + 1;
+  uint32_t* flags = hist + kHistCopies * 256;
+  __shared__ uint32_t s_bucket_info[2];
+  __shared__ int s_iscr[NW];
+
+  const int tid = threadIdx.x;
+  const int row = blockIdx.x;
+  grid_dependency_wait();   // the kept lists come from the block selection
+
+  const int b = row / a.Hkv;
+  int Tb = a.seq_lens ? a.seq_lens[b] : a.T;
+  Tb = Tb < 0 ? 0 : (Tb > a.T ? a.T : Tb);
+  const int nbr = (Tb + kBlock - 1) / kBlock;
+  const int c0 = min(a.n_sink, nbr);
+  const int c1 = max(c0, nbr - a.n_local);
+  const int gpb = kBlock / a.group_size;
+  const uint32_t all = gpb == 32 ? 0xffffffffu : (1u << gpb) - 1u;
+  const int32_t* kept = a.kept + static_cast<int64_t>(row) * a.max_kept;
+  int32_t* out = a.kept_groups + static_cast<int64_t>(row) * a.max_kept;
+  const int count = max(0, min(a.kept_count[row], a.max_kept));
+  // the dynamic entries sit between the sink prefix and the local suffix
+  int kdyn = max(0, count - c0 - (nbr - c1));
+  if (kdyn * gpb > a.max_cand) {   // more dynamic entries than k_max: not a kept list
+    report(a.status, BSA_DEV_BAD_KEPT);
+    kdyn = a.max_cand / gpb;
+  }
+  for (int e = tid; e < kdyn; e += NT) {
+    const int j = kept[c0 + e];
+    const bool ok = j >= c0 && j < c1;
+    if (!ok) report(a.status, BSA_DEV_BAD_KEPT);
+    ids[e] = ok ? j : -1;
+  }
+  __syncthreads();
+  // groups of the last block that start past the sequence do not exist; only the
+  // last dynamic entry can be that block
+  int ncand = kdyn * gpb;
+  if (kdyn > 0 && ids[kdyn - 1] == nbr - 1)
+    ncand -= gpb - (Tb - (nbr - 1) * kBlock + a.group_size - 1) / a.group_size;
+  const int64_t ngr = static_cast<int64_t>(a.nb_max) * gpb;
+  const float* Sg = a.group_scores + static_cast<int64_t>(row) * ngr;
+  for (int t = tid; t < ncand; t += NT) {
+    const int j = ids[t / gpb];
+    // a rejected entry takes part with the lowest priority and is dropped below
+    keys[skew(t)] = j >= 0 ? order_key(Sg[static_cast<int64_t>(j) * gpb + t % gpb]) : 0xffffffffu;
+  }
+  const int nflag_words = (ncand + 31) / 32;
+  for (int w = tid; w < nflag_words; w += NT) flags[w] = 0u;
+  __syncthreads();
+
+  const int kg = min(a.k_groups, ncand);
+  if (kg == ncand) {
+    for (int t = tid; t < ncand; t += NT) atomicOr(&flags[t >> 5], 1u << (t & 31));
+  } else if (kg > 0) {
+    int rem = kg;
+    const uint32_t prefix = radix_kth<NT>(keys, ncand, rem, hist, s_bucket_info);
+    const int E = (ncand + NT - 1) / NT;
+    const int seg0 = min(ncand, tid * E), seg1 = min(ncand, seg0 + E);
+    int neq = 0;
+    for (int t = seg0; t < seg1; ++t) neq += (keys[skew(t)] == prefix);
+    int tot_eq;
+    int eq_base = block_exscan<NT>(neq, s_iscr, tot_eq);
+    for (int t = seg0; t < seg1; ++t) {
+      const uint32_t k = keys[skew(t)];
+      bool in = k < prefix;
+      if (k == prefix) in = (eq_base++ < rem);
+      if (in) atomicOr(&flags[t >> 5], 1u << (t & 31));
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < a.max_kept; e += NT) {
+    uint32_t m = 0u;
+    if (e < c0 || (e >= c0 + kdyn && e < count)) {
+      m = all;   // sink and local blocks stay whole
+    } else if (e < c0 + kdyn && ids[e - c0] >= 0) {
+      for (int k = 0; k < gpb; ++k) {
+        const int t = (e - c0) * gpb + k;
+        if (t < ncand && ((flags[t >> 5] >> (t & 31)) & 1u)) m |= 1u << k;
+      }
+    }
+    out[e] = static_cast<int32_t>(m);
+  }
 }
 
 // Writes `v` into slot `slot` of the array `box` of every CTA of the cluster. The
@@ -733,6 +840,20 @@ cudaError_t launch_cluster(const SelectArgs& a, int rows, int max_nc, cudaStream
 }
 
 }  // namespace
+
+cudaError_t launch_select_groups(const GroupSelectArgs& a, cudaStream_t s) {
+  const int rows = a.B * a.Hkv;
+  if (rows <= 0) return cudaSuccess;
+  const size_t nflag_words = (a.max_cand + 31) / 32;
+  size_t smem = static_cast<size_t>(a.max_kept) * 4 + (static_cast<size_t>(skew(a.max_cand)) + 1) * 4 +
+                kHistCopies * 256 * 4 + (nflag_words + 1) * 4;
+  smem = (smem + 15) & ~static_cast<size_t>(15);
+  cudaError_t e = cudaFuncSetAttribute(select_groups_kernel<256>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(select_groups_kernel<256>, dim3(rows), dim3(256), smem, s, a);
+}
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
   int rows, max_nc;

@@ -122,6 +122,20 @@ typedef struct {
   const int32_t* key_pos;   /* prefill with segment > 0: device [B, Hkv, T] original position
                                of the key at each permuted position (bsa_pbs_permute's output);
                                bsa_prefill masks the keys of the query's own segment by it */
+  int32_t group_size;       /* decode only: 0, or 16, 32 or 64 for two-level routing (HGA,
+                               "Hierarchical Global Attention", Central mechanism §2): the
+                               dynamically selected blocks are refined to their best groups
+                               of group_size tokens. A group's score is the max of its tokens'
+                               index scores; the k_groups best groups of the dynamic blocks
+                               (score descending, lower group id on ties) are kept; sink and
+                               local blocks stay whole. k_max * 64 / group_size <= 8192. */
+  int32_t k_groups;         /* cap on the kept groups (group_size > 0) */
+  float* group_scores;      /* group_size > 0: device [B, Hkv, nb * 64 / group_size] fp32,
+                               written by bsa_score_blocks (groups past a sequence: -inf) */
+  int32_t* kept_groups;     /* group_size > 0: device [B, Hkv, max_kept] int32, written by
+                               bsa_select_top_p: bit k of entry e set when group k of kept
+                               block e is attended (all bits for sink and local blocks, 0 for
+                               unused slots); read by bsa_decode */
 } bsa_problem_t;
 
 /* Length of one kept list: decode n_sink + n_local + k_max; prefill

@@ -332,3 +332,94 @@ def compare_pbs_rows(w, inputs, pbs, b, g, rows, seg):
     for i, ref in refs.items():
         _check_prefill_block(w, o32, lse, b, g, i, ref, summary)
     return summary
+
+
+# ------------------------------------------------------------------ two-level (HGA) decode rows
+GROUP_TIE_REL = 1e-5   # group scores this close (relative) may rank either way
+
+
+def group_verdict(Sg, cand, groups_ref, groups_dev, k_groups, tol=GROUP_TIE_REL):
+    """'exact' | 'tie' | 'mismatch: ...' for the device's kept groups: the right
+    number of candidate groups, and any difference to the oracle's choice lies at
+    the boundary score (within tol relative)."""
+    Dd, Do = set(groups_dev), set(groups_ref)
+    if not Dd <= set(cand):
+        return f"mismatch: groups outside the candidates {sorted(Dd - set(cand))}"
+    if len(Dd) != min(k_groups, len(cand)):
+        return f"mismatch: {len(Dd)} groups on the device, {min(k_groups, len(cand))} expected"
+    if Dd == Do:
+        return "exact"
+    sb = min(Sg[c] for c in Do)
+    bad = [c for c in Dd ^ Do if abs(Sg[c] - sb) > tol * max(1.0, abs(sb))]
+    return "tie" if not bad else f"mismatch: groups {sorted(Dd ^ Do)} differ (boundary {sb})"
+
+
+def compare_hga_rows(w, inputs, step, rows, gs, k_groups):
+    """Compare a finished two-level DecodeStep with the HGA oracle on (b, g) rows:
+    block scores, group scores, kept blocks (tie rule on mass), kept groups (tie rule
+    on score), the masks of the always-visible entries, attention."""
+    from oracle import hga_oracle as H
+    G = w.G
+    gpb = 64 // gs
+    kept, cnt = step.kept.cpu(), step.kept_count.cpu()
+    scores, gsc = step.scores.cpu(), step.group_scores.cpu()
+    masks = step.kept_groups.cpu()
+    o, o32, lse = step.o.cpu(), step.o_f32.cpu(), step.lse.cpu()
+    assert bf16_is_rne_of_f32(o, o32), "bf16 output is not RNE(fp32 output)"
+    summary = {"rows": 0, "ties": 0, "group_ties": 0, "max_abs": 0.0, "rel_l2": 0.0,
+               "lse_abs": 0.0, "score_rel": 0.0, "groups": 0}
+    pt = inputs.get("page_table")
+    for (b, g) in rows:
+        T_b = int(inputs["seq_lens"][b])
+        q_g = f64(inputs["q"][b, g * G:(g + 1) * G])
+        _, qi_g, hw = index_heads(inputs, w, b, g, (slice(None),))
+        ki_g = f64(inputs["k_idx"][b, g, :T_b])
+        ids = np.arange(T_b)
+        K_g = f64(logical_rows(inputs["K"], pt, b, g, ids))
+        V_g = f64(logical_rows(inputs["V"], pt, b, g, ids))
+        args = (q_g, qi_g, ki_g, K_g, V_g, T_b, hw, 1.0 / math.sqrt(w.r), 1.0 / math.sqrt(w.d),
+                w.n_sink, w.n_local, w.p, w.k_max, gs, k_groups, w.k_min)
+        ref = H.hga_decode_row(*args)
+        nb = len(ref["S"])
+        if nb:
+            S_dev = scores[b, g, :nb].double().numpy()
+            rel = np.max(np.abs(S_dev - ref["S"]) / np.maximum(1.0, np.abs(ref["S"])))
+            ng = len(ref["Sg"])
+            Sg_dev = gsc[b, g, :ng].double().numpy()
+            grel = np.max(np.abs(Sg_dev - ref["Sg"]) / np.maximum(1.0, np.abs(ref["Sg"])))
+            summary["score_rel"] = max(summary["score_rel"], float(rel), float(grel))
+            assert rel <= SCORE_REL, f"row {(b, g)}: block score rel err {rel}"
+            assert grel <= SCORE_REL, f"row {(b, g)}: group score rel err {grel}"
+            tail = gsc[b, g, ng:nb * gpb]
+            assert bool(torch.all(tail == float("-inf"))), "groups past the end are not -inf"
+        c = int(cnt[b, g])
+        kd = kept[b, g, :c].tolist()
+        v = selection_verdict(ref["sel"], kd, w.p)
+        assert not v.startswith("mismatch"), f"row {(b, g)}: {v}"
+        if v == "tie":
+            summary["ties"] += 1
+            ref = H.hga_decode_row(*args, kept_override=kd)
+        m = [int(x) & 0xffffffff for x in masks[b, g].tolist()]
+        full = (1 << gpb) - 1
+        R = set(ref["sel"].reserved)
+        gdev = []
+        for e, j in enumerate(kd):
+            if j in R:
+                assert m[e] == full, f"row {(b, g)}: always-visible block {j} mask {m[e]:#x}"
+            else:
+                assert m[e] >> gpb == 0, f"row {(b, g)}: mask {m[e]:#x} has bits past the block"
+                gdev += [j * gpb + k for k in range(gpb) if (m[e] >> k) & 1]
+        assert all(x == 0 for x in m[c:]), f"row {(b, g)}: masks past the count are not 0"
+        gv = group_verdict(ref["Sg"], ref["cand"], ref["groups"], gdev, k_groups)
+        assert not gv.startswith("mismatch"), f"row {(b, g)}: {gv}"
+        if gv == "tie":
+            summary["group_ties"] += 1
+            ref = H.hga_decode_row(*args, kept_override=kd, groups_override=gdev)
+        errs = attention_errors(o32[b, g * G:(g + 1) * G].double().numpy(), None,
+                                lse[b, g * G:(g + 1) * G].double().numpy(), ref["o"], ref["lse"])
+        check_attention(errs, f"row {(b, g)}")
+        for k_ in ("max_abs", "rel_l2", "lse_abs"):
+            summary[k_] = max(summary[k_], errs[k_])
+        summary["rows"] += 1
+        summary["groups"] += len(gdev)
+    return summary

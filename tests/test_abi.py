@@ -69,6 +69,9 @@ def test_workspace_size_host_only(lib):
     (dict(p=float("nan")), bsa.BSA_ERR_INVALID_ARG),
     (dict(B=0), bsa.BSA_ERR_INVALID_ARG),
     (dict(T=64 * 40000), bsa.BSA_ERR_UNSUPPORTED),
+    (dict(group_size=8, k_groups=4), bsa.BSA_ERR_UNSUPPORTED),     # groups of 16, 32, 64
+    (dict(group_size=16, k_groups=-1), bsa.BSA_ERR_INVALID_ARG),
+    (dict(group_size=16, k_groups=4, k_max=4096), bsa.BSA_ERR_UNSUPPORTED),   # > 8192 groups
 ])
 def test_invalid_problems_rejected(lib, kw, code):
     out = ctypes.c_size_t(0)
@@ -120,3 +123,21 @@ def test_qcache_entry_points_reject_on_host(lib):
                                            None) == bsa.BSA_ERR_INVALID_ARG
     assert lib.bsa_score_blocks_q(ctypes.byref(p), None, _qcache(), 0x50000, None,
                                   None) == bsa.BSA_ERR_INVALID_ARG
+
+
+def test_group_routing_rejects_on_host(lib):
+    """Two-level routing: decode only, and each step needs its group buffers."""
+    pf = _prob(phase=bsa.PHASE_PREFILL, group_size=16, k_groups=4).c()
+    out = ctypes.c_size_t(0)
+    assert lib.bsa_workspace_size(ctypes.byref(pf), bsa.OP_PREFILL,
+                                  ctypes.byref(out)) == bsa.BSA_ERR_INVALID_ARG
+    p = _prob(group_size=16, k_groups=4).c()          # group_scores / kept_groups null
+    assert lib.bsa_score_blocks(ctypes.byref(p), 0x40000, _kcache(), 0x50000, None,
+                                None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_score_blocks_q(ctypes.byref(p), 0x40000, _qcache(), 0x50000, None,
+                                  None) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_select_top_p(ctypes.byref(p), 0x50000, 0x60000, 0x70000, None,
+                                None) == bsa.BSA_ERR_INVALID_ARG
+    p.group_scores = 0x80000                          # kept_groups still null
+    assert lib.bsa_select_top_p(ctypes.byref(p), 0x50000, 0x60000, 0x70000, None,
+                                None) == bsa.BSA_ERR_INVALID_ARG
