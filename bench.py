@@ -396,6 +396,8 @@ def run_ours(args, world, rank, local):
             extras["decode_fp4"] = time_decode(wd, xd, dprob, dstep, qc, K_c, V_c, "fp4", dev,
                                                world, args.extra_steps, peaks)
             del qc
+            extras["decode_hga"] = time_hga(wd, xd, k_idx_c, K_c, V_c, dev, world,
+                                            args.extra_steps, peaks, 16, 2 * wd.k_max)
             del xd, dstep, K_c, V_c, k_idx_c
             torch.cuda.empty_cache()
             for key, name in (("decode_c2", "decode_b8_h32_t32k_paged"),
@@ -479,6 +481,31 @@ def time_decode(w, xd, prob, step, k_idx, K, V, index_cache, dev, world, steps, 
             "tokens_per_s": world * w.B / (ms / 1e3), "hbm_gbs": gbs,
             "hbm_frac": gbs / peaks["hbm_gbs"], "bytes_per_step": by["step"], "steps": steps,
             "device_status": st}
+
+
+def time_hga(w, xd, k_idx, K, V, dev, world, steps, peaks, gs, k_groups):
+    """Decode with two-level routing (HGA): the kept blocks' best k_groups groups of gs
+    tokens. Algorithmic bytes: every index key, q and the outputs, and K and V of
+    the copied 16-token quarters (whole always-visible blocks, kept groups of the
+    others); the intermediate block and group scores are not counted."""
+    prob = bsa.problem_for(w, seq_lens=xd["seq_lens"], head_w=xd["head_w"])
+    prob.group_size, prob.k_groups = gs, k_groups
+    step = bsa.DecodeStep(prob, device=dev, keep_f32=False)
+    out = time_decode(w, xd, prob, step, k_idx, K, V, "bf16", dev, world, steps, peaks)
+    by = decode_bytes(w, step.kept_count, xd["seq_lens"], "bf16")
+    m = step.kept_groups.to(torch.int64).cpu()
+    quarters = sum(int(((m >> q4) & 1).sum()) for q4 in range(4)) if gs == 16 else None
+    if quarters is not None:
+        kv = quarters * 16 * w.d * 2 * 2
+        step_bytes = by["step"] - by["kv"] + kv
+        gbs = step_bytes / (out["ms"] / 1e3) / 1e9
+        out.update({"bytes_per_step": step_bytes, "hbm_gbs": gbs,
+                    "hbm_frac": gbs / peaks["hbm_gbs"], "kv_tokens": quarters * 16})
+    out.update({"group_size": gs, "k_groups": k_groups,
+                "kept_blocks": int(step.kept_count.sum())})
+    del step
+    torch.cuda.empty_cache()
+    return out
 
 
 def time_decode_workload(name, rank, dev, world, steps, peaks):

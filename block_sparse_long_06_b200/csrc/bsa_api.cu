@@ -263,7 +263,8 @@ bsa_status_t bsa_score_blocks(const bsa_problem_t* p, const void* q_idx, bsa_cac
   bsa_status_t st = check_problem(p);
   if (st != BSA_OK) return st;
   if (q_idx == nullptr || block_scores == nullptr || !aligned16(q_idx)) return BSA_ERR_INVALID_ARG;
-  if (p->group_size > 0 && p->group_scores == nullptr) return BSA_ERR_INVALID_ARG;
+  if (p->group_size > 0 && (p->group_scores == nullptr || !aligned16(p->group_scores)))
+    return BSA_ERR_INVALID_ARG;
   if ((st = check_cache(k_idx, p, p->r, false)) != BSA_OK) return st;
   const int num_sms = num_sms_current();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -340,7 +341,8 @@ bsa_status_t bsa_score_blocks_q(const bsa_problem_t* p, const void* q_idx, bsa_q
   if (st != BSA_OK) return st;
   if (p->phase != BSA_PHASE_DECODE) return BSA_ERR_UNSUPPORTED;
   if (q_idx == nullptr || block_scores == nullptr || !aligned16(q_idx)) return BSA_ERR_INVALID_ARG;
-  if (p->group_size > 0 && p->group_scores == nullptr) return BSA_ERR_INVALID_ARG;
+  if (p->group_size > 0 && (p->group_scores == nullptr || !aligned16(p->group_scores)))
+    return BSA_ERR_INVALID_ARG;
   if ((st = check_qcache(k_idx, p)) != BSA_OK) return st;
   bsa::ScoreDecodeArgs a{};
   a.q_idx = q_idx;
@@ -440,17 +442,18 @@ bsa_status_t bsa_decode(const bsa_problem_t* p, const void* q, bsa_cache_t k, bs
   if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return BSA_ERR_WORKSPACE;
   if (p->group_size > 0 && p->kept_groups == nullptr) return BSA_ERR_INVALID_ARG;
-  CUtensorMap tk, tv, tk16, tv16;
-  if (!make_map(&tk, k.base, k.extent / p->d, p->d, false) ||
-      !make_map(&tv, v.base, v.extent / p->d, p->d, false))
+  bsa::DecodeMaps maps;
+  if (!make_map(&maps.k, k.base, k.extent / p->d, p->d, false) ||
+      !make_map(&maps.v, v.base, v.extent / p->d, p->d, false))
     return cuda_fail(cudaErrorInvalidValue);
   if (p->group_size > 0) {
-    if (!make_map(&tk16, k.base, k.extent / p->d, p->d, false, 16) ||
-        !make_map(&tv16, v.base, v.extent / p->d, p->d, false, 16))
+    if (!make_map(&maps.k16, k.base, k.extent / p->d, p->d, false, 16) ||
+        !make_map(&maps.v16, v.base, v.extent / p->d, p->d, false, 16))
       return cuda_fail(cudaErrorInvalidValue);
   } else {
-    tk16 = tk;   // not read: every kept block is copied whole
-    tv16 = tv;
+    // not read: every kept block is copied whole
+    maps.k16 = maps.k;
+    maps.v16 = maps.v;
   }
   bsa::DecodeArgs a{};
   a.q = q;
@@ -477,8 +480,7 @@ bsa_status_t bsa_decode(const bsa_problem_t* p, const void* q, bsa_cache_t k, bs
   a.scale_log2 = attn_scale_of(p) * 1.4426950408889634f;
   a.kept_groups = p->group_size > 0 ? p->kept_groups : nullptr;
   a.group_size = p->group_size;
-  cudaError_t e = bsa::launch_decode(a, tk, tv, tk16, tv16, pl.units, num_sms,
-                                     static_cast<cudaStream_t>(stream));
+  cudaError_t e = bsa::launch_decode(a, maps, pl.units, num_sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BSA_OK : cuda_fail(e);
 }
 

@@ -160,10 +160,13 @@ cudaError_t launch_quantize_index(const QuantArgs& a, int num_sms, cudaStream_t 
 cudaError_t launch_score_prefill(const ScorePrefillArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_select_groups(const GroupSelectArgs& a, cudaStream_t s);
-// tk16 / tv16: the same caches with 16-row boxes (copies of partly kept blocks).
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const CUtensorMap& tk16, const CUtensorMap& tv16, int num_units,
-                          int num_sms, cudaStream_t s);
+// Tensor maps of the K and V caches for decode: 64-row boxes (whole blocks) and
+// 16-row boxes (kept 16-token quarters under two-level routing).
+struct DecodeMaps {
+  CUtensorMap k, v, k16, v16;
+};
+cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, int num_units, int num_sms,
+                          cudaStream_t s);
 cudaError_t launch_v_to_f16(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, const CUtensorMap& tq, const CUtensorMap& tk,
                               const CUtensorMap& tv16, int* unit_counter, int num_sms,

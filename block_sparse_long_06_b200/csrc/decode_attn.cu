@@ -19,11 +19,14 @@
 //  * at the end of a unit the four warps' (m, l, O) are merged in shared memory
 //    and written as one partial; the merge kernel combines the splits of a row
 //    with their log-sum-exp weights and writes o (bf16), o_f32 and lse.
+//  * a stage holds four 16-token slots, consumer warp w attends slot w; the
+//    producer publishes each slot's first token (or -1) and whether the stage is
+//    the last of its unit. Without group masks a stage is one kept block.
 //  * two-level routing (HGA, Central mechanism §2): each kept entry carries a
-//    bitmask of its kept token groups. A block with every group kept is copied as
-//    above; otherwise only the 16-token quarters of its kept groups are copied
-//    (16-row boxes at the same swizzled offsets), and a consumer warp whose
-//    quarter was not copied skips the block.
+//    bitmask of its kept token groups, and the producer packs the 16-token
+//    quarters of the kept groups of consecutive entries densely into the slots
+//    (16-row boxes at the slots' swizzled offsets), so a stage carries four
+//    quarters of useful work whatever the groups kept.
 #include "bsa_common.cuh"
 #include "bsa_internal.h"
 
@@ -48,7 +51,8 @@ struct DecodeSmem {
   static constexpr int kComb = kConsumerWarps * (NT * 8) * D * 4;   // partial O per warp
   static constexpr int kStats = kConsumerWarps * (NT * 8) * 2 * 4;  // m, l per warp
   static constexpr int kBars = 2 * DecodeCfg<D>::kStages * 8;
-  static constexpr int kInfo = DecodeCfg<D>::kStages * 4;
+  static constexpr int kInfoW = 5;   // per stage: first token of slots 0..3, last-of-unit flag
+  static constexpr int kInfo = DecodeCfg<D>::kStages * kInfoW * 4;
   static constexpr int kTotal = kRing + kComb + kStats + kBars + kInfo + 1024;  // + alignment
 };
 
@@ -129,7 +133,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tmv16);
       }
     }
-    uint32_t it = 0;
+    constexpr int kW = Sm::kInfoW;
+    const bool packed = a.kept_groups != nullptr;
+    uint32_t it = 0;   // stages issued
     bool ok_all = true;
     for (int unit = blockIdx.x; unit < num_units && ok_all; unit += gridDim.x) {
       const int row = unit / a.splits, sp = unit % a.splits;
@@ -138,6 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int e0 = sp * a.split_len, e1 = min(cnt, e0 + a.split_len);
       const int Tb = seq_len(a, b);
       const int nb = (Tb + kBlock - 1) / kBlock;
+      bool open = false;   // packed: a stage is being filled (lane 0)
+      int fill = 0;        // packed: its slots in use
       for (int base = e0; base < e1 && ok_all; base += 32) {
         const int e = base + lane;
         int blk = -1, qm = 15;   // qm: 16-token quarters to copy and attend
@@ -149,57 +157,86 @@ __global__ void __launch_bounds__(kThreads, 1)
             rk = tile_row(a.k, b, g, blk, rows, D);
             rv = tile_row(a.v, b, g, blk, rows, D);
             if (rk < 0 || rv < 0) report(a.status, BSA_DEV_BAD_PAGE);
-            if (a.kept_groups != nullptr) {
+            if (packed) {
               const uint32_t gm = static_cast<uint32_t>(
                   a.kept_groups[static_cast<int64_t>(row) * a.max_kept + e]);
               qm = 0;
 #pragma unroll
               for (int q = 0; q < 4; ++q) qm |= static_cast<int>((gm >> (q * 16 / a.group_size)) & 1u) << q;
-              // a partly kept block: only its quarters that hold tokens
-              if (qm != 15) qm &= (1 << ((rows + 15) / 16)) - 1;
+              qm &= (1 << ((rows + 15) / 16)) - 1;   // quarters that hold tokens
             }
           } else {
             report(a.status, BSA_DEV_BAD_KEPT);
           }
         }
         const int n_here = min(32, e1 - base);
-        for (int q = 0; q < n_here; ++q, ++it) {
+        for (int q = 0; q < n_here; ++q) {
           const int blk_q = __shfl_sync(0xffffffffu, blk, q);
           const int64_t rk_q = __shfl_sync(0xffffffffu, rk, q);
           const int64_t rv_q = __shfl_sync(0xffffffffu, rv, q);
           const int qm_q = __shfl_sync(0xffffffffu, qm, q);
           if (lane == 0) {
-            const int s = it % S;
-            if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
-              report(a.status, BSA_DEV_TIMEOUT);
-              ok_all = false;
-            } else {
-              const bool ok = rk_q >= 0 && rv_q >= 0 && qm_q != 0;
-              sinfo[s] = ok ? (blk_q << 4) | qm_q : -1;
-              unsigned char* st = ring + s * Cfg::kStageBytes;
-              if (ok && qm_q == 15) {
-                mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
+            const bool ok = rk_q >= 0 && rv_q >= 0;
+            if (!packed) {
+              // one kept block per stage
+              const int s = it % S;
+              if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
+                report(a.status, BSA_DEV_TIMEOUT);
+                ok_all = false;
+              } else {
 #pragma unroll
-                for (int x = 0; x < Cfg::kBoxes; ++x) {
-                  tma_load_2d(st + x * 8192, &tmk, x * 64, static_cast<int32_t>(rk_q), &full[s]);
-                  tma_load_2d(st + Cfg::kTileBytes + x * 8192, &tmv, x * 64,
-                              static_cast<int32_t>(rv_q), &full[s]);
-                }
-              } else if (ok) {
-                // kept quarters only: 16 rows x 64 dims per box, 2 KB apart in the tile
-                mbar_arrive_expect_tx(&full[s], __popc(qm_q) * Cfg::kStageBytes / 4);
-                for (int q4 = 0; q4 < 4; ++q4) {
-                  if (!((qm_q >> q4) & 1)) continue;
+                for (int w = 0; w < 4; ++w) sinfo[s * kW + w] = ok ? blk_q * kBlock + 16 * w : -1;
+                sinfo[s * kW + 4] = base + q == e1 - 1;
+                unsigned char* st = ring + s * Cfg::kStageBytes;
+                if (ok) {
+                  mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
 #pragma unroll
                   for (int x = 0; x < Cfg::kBoxes; ++x) {
-                    tma_load_2d(st + x * 8192 + q4 * 2048, &tmk16, x * 64,
-                                static_cast<int32_t>(rk_q + 16 * q4), &full[s]);
-                    tma_load_2d(st + Cfg::kTileBytes + x * 8192 + q4 * 2048, &tmv16, x * 64,
-                                static_cast<int32_t>(rv_q + 16 * q4), &full[s]);
+                    tma_load_2d(st + x * 8192, &tmk, x * 64, static_cast<int32_t>(rk_q), &full[s]);
+                    tma_load_2d(st + Cfg::kTileBytes + x * 8192, &tmv, x * 64,
+                                static_cast<int32_t>(rv_q), &full[s]);
                   }
+                } else {
+                  mbar_arrive(&full[s]);
                 }
-              } else {
-                mbar_arrive(&full[s]);
+                ++it;
+              }
+            } else {
+              // the entry's kept quarters go to the next free slots, one 16-row copy
+              // each (issuing whole runs through run-length-dependent branches measured
+              // slower); a full stage is handed over once it is known not to be the
+              // unit's last
+              for (int q4 = 0; q4 < 4 && ok && ok_all; ++q4) {
+                if (!((qm_q >> q4) & 1)) continue;
+                if (open && fill == 4) {
+                  const int s = (it - 1) % S;
+                  sinfo[s * kW + 4] = 0;
+                  mbar_arrive(&full[s]);
+                  open = false;
+                }
+                if (!open) {
+                  const int s = it % S;
+                  if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
+                    report(a.status, BSA_DEV_TIMEOUT);
+                    ok_all = false;
+                    break;
+                  }
+                  ++it;
+                  open = true;
+                  fill = 0;
+                }
+                const int s = (it - 1) % S;
+                sinfo[s * kW + fill] = blk_q * kBlock + 16 * q4;
+                unsigned char* st = ring + s * Cfg::kStageBytes + fill * 2048;
+                mbar_expect_tx(&full[s], Cfg::kStageBytes / 4);
+#pragma unroll
+                for (int x = 0; x < Cfg::kBoxes; ++x) {
+                  tma_load_2d(st + x * 8192, &tmk16, x * 64, static_cast<int32_t>(rk_q + 16 * q4),
+                              &full[s]);
+                  tma_load_2d(st + Cfg::kTileBytes + x * 8192, &tmv16, x * 64,
+                              static_cast<int32_t>(rv_q + 16 * q4), &full[s]);
+                }
+                ++fill;
               }
             }
           }
@@ -207,6 +244,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok_all) break;
         }
       }
+      // packed: close the unit's last stage (an empty one when no quarter was kept)
+      if (packed && e1 > e0 && ok_all && lane == 0) {
+        if (!open) {
+          const int s = it % S;
+          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
+            report(a.status, BSA_DEV_TIMEOUT);
+            ok_all = false;
+          } else {
+            ++it;
+            open = true;
+            fill = 0;
+          }
+        }
+        if (open) {
+          const int s = (it - 1) % S;
+          for (int w = fill; w < 4; ++w) sinfo[s * kW + w] = -1;
+          sinfo[s * kW + 4] = 1;
+          mbar_arrive(&full[s]);
+        }
+      }
+      ok_all = __shfl_sync(0xffffffffu, ok_all ? 1 : 0, 0) != 0;
     }
     // drain: wait until the consumers released every stage we filled (bounded)
     if (lane == 0) {
@@ -256,19 +314,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
     }
 
-    for (int e = e0; e < e1 && alive; ++e, ++it) {
+    // stages of this unit until the one marked last (none for an empty unit)
+    for (bool last = e1 <= e0; !last && alive; ++it) {
       const int s = it % S;
       if (!mbar_wait(&full[s], (it / S) & 1)) {
         if (lane == 0) report(a.status, BSA_DEV_TIMEOUT);
         alive = false;
         break;
       }
-      const int info = sinfo[s];
-      const int blk = info >> 4;   // -1 when nothing was copied
-      if (info >= 0 && ((info >> warp) & 1)) {
+      last = sinfo[s * Sm::kInfoW + 4] != 0;
+      const int tok0 = sinfo[s * Sm::kInfoW + warp];   // first token of this warp's slot
+      if (tok0 >= 0) {
         const uint32_t kb = smem_u32(ring + s * Cfg::kStageBytes);
         const uint32_t vb = kb + Cfg::kTileBytes;
-        const int valid = Tb - blk * kBlock - 16 * warp;  // tokens of this warp that exist
+        const int valid = Tb - tok0;  // tokens of this warp's slot that exist
         // ---- S^T = K_w Q^T
         float sc[NT][4];
 #pragma unroll
@@ -456,8 +515,8 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a) {
 
 template <int D, int NT>
 cudaError_t launch_dn(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                      const CUtensorMap& tk16, const CUtensorMap& tv16, int num_units,
-                      int num_sms, cudaStream_t s) {
+                      const CUtensorMap& tk16, const CUtensorMap& tv16, int num_units, int num_sms,
+                      cudaStream_t s) {
   const int smem = DecodeSmem<D, NT>::kTotal;
   auto kern = decode_attn_kernel<D, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -492,16 +551,15 @@ void decode_split_plan(int rows, int max_kept, int num_sms, int* splits, int* sp
   *splits = max_kept > 0 ? (max_kept + best_len - 1) / best_len : 1;
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const CUtensorMap& tk16, const CUtensorMap& tv16, int num_units,
-                          int num_sms, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, int num_units, int num_sms,
+                          cudaStream_t s) {
   const int NT = a.G > 8 ? 2 : 1;
   if (a.d == 128) {
-    return NT == 1 ? launch_dn<128, 1>(a, tk, tv, tk16, tv16, num_units, num_sms, s)
-                   : launch_dn<128, 2>(a, tk, tv, tk16, tv16, num_units, num_sms, s);
+    return NT == 1 ? launch_dn<128, 1>(a, m.k, m.v, m.k16, m.v16, num_units, num_sms, s)
+                   : launch_dn<128, 2>(a, m.k, m.v, m.k16, m.v16, num_units, num_sms, s);
   }
-  return NT == 1 ? launch_dn<64, 1>(a, tk, tv, tk16, tv16, num_units, num_sms, s)
-                 : launch_dn<64, 2>(a, tk, tv, tk16, tv16, num_units, num_sms, s);
+  return NT == 1 ? launch_dn<64, 1>(a, m.k, m.v, m.k16, m.v16, num_units, num_sms, s)
+                 : launch_dn<64, 2>(a, m.k, m.v, m.k16, m.v16, num_units, num_sms, s);
 }
 
 }  // namespace bsa

@@ -136,7 +136,8 @@ BSA_DEVFN bool block_offset(const CacheView& c, int b, int g, int blk, int rows,
   return off >= 0 && off + static_cast<int64_t>(rows) * kR <= c.extent;
 }
 
-template <int NT, int KF>
+// GRP: also write the maxima of the token groups (two-level routing).
+template <int NT, int KF, bool GRP>
 __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecodeArgs a) {
   using SM = ScoreSmem<KF>;
   constexpr int kStages = SM::kStages, kStageBytes = SM::kStageBytes, kBlockBytes = SM::kBlockBytes;
@@ -309,7 +310,7 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
     if (j < a.nb_max) {
       float* out = a.scores + static_cast<int64_t>(in.row) * a.nb_max + j;
       const int valid = in.Tb - j * kBlock;  // tokens of this block that exist
-      const int gpb = a.group_size > 0 ? kBlock / a.group_size : 0;
+      const int gpb = GRP ? kBlock / a.group_size : 0;
       float* gout = gpb ? a.group_scores + (static_cast<int64_t>(in.row) * a.nb_max + j) * gpb : nullptr;
       if (valid <= 0 || !(in.ok & (1u << warp))) {
         if (lane == 0) {
@@ -320,7 +321,10 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
       } else {
         const unsigned char* blk = ring + s * kStageBytes + warp * kBlockBytes;
         float mx = 0.f;
-        float gm[4];   // this lane's token score of each 16-token group (-inf past the end)
+        // two-level routing: the max of each 16-token group (tile mt) as the bits of a
+        // non-negative float (the scores are >= 0, so integer order is float order),
+        // -1 when the group holds no token of the sequence
+        int gbits[4] = {-1, -1, -1, -1};
         const bool odd = tig & 1;
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
@@ -360,26 +364,22 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
           const int tok = odd ? r1 : r0;
           if constexpr (KF != 0) keep *= scale_lut[blk[kBlock * 8 + tok] & 0x7Fu];   // token scale
           if (tok < valid) mx = fmaxf(mx, keep);
-          gm[mt] = tok < valid ? keep : -INFINITY;
+          if constexpr (GRP) gbits[mt] = __reduce_max_sync(0xffffffffu, tok < valid ? __float_as_int(keep) : -1);
         }
-        if (gpb) {
-          // group maxima (HGA, Central mechanism §2: group summaries, here the max of
-          // the group's token scores): a transposing butterfly reduces the four
-          // 16-token groups in 6 shuffles; lane 8m ends with group m.
-          const bool h16 = lane & 16, h8 = lane & 8;
-          float k0 = h16 ? gm[2] : gm[0], k1 = h16 ? gm[3] : gm[1];
-          k0 = fmaxf(k0, __shfl_xor_sync(0xffffffffu, h16 ? gm[0] : gm[2], 16));
-          k1 = fmaxf(k1, __shfl_xor_sync(0xffffffffu, h16 ? gm[1] : gm[3], 16));
-          float gk = h8 ? k1 : k0;
-          gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8));
-          gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, 4));
-          gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, 2));
-          gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, 1));
-          if (gpb <= 2) gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, 8));    // 32-token groups
-          if (gpb == 1) gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, 16));   // one group
-          const int step = 32 / gpb;   // lane of group m: m * step
-          if ((lane & (step - 1)) == 0)
-            gout[lane / step] = gk == -INFINITY ? -INFINITY : a.idx_scale * (kscale * gk);
+        if (GRP && lane == 0) {
+          // group summaries (HGA, Central mechanism §2), here the max of the group's
+          // token scores: 16-token groups are the tiles, larger ones their maxima
+          const float sc = a.idx_scale * kscale;
+          auto val = [sc](int bits) { return bits < 0 ? -INFINITY : sc * __int_as_float(bits); };
+          if (gpb == 4) {
+            *reinterpret_cast<float4*>(gout) =
+                make_float4(val(gbits[0]), val(gbits[1]), val(gbits[2]), val(gbits[3]));
+          } else if (gpb == 2) {
+            *reinterpret_cast<float2*>(gout) =
+                make_float2(val(max(gbits[0], gbits[1])), val(max(gbits[2], gbits[3])));
+          } else {
+            *gout = val(max(max(gbits[0], gbits[1]), max(gbits[2], gbits[3])));
+          }
         }
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
@@ -402,7 +402,9 @@ cudaError_t launch_fmt(const ScoreDecodeArgs& a, int num_sms, cudaStream_t s) {
   const int smem = ScoreSmem<KF>::kTotal;
   int64_t ctas = static_cast<int64_t>(num_sms) * ScoreSmem<KF>::kCtasPerSm;
   if (ctas > a.total_items) ctas = a.total_items;
-  auto kern = (a.G > 8) ? score_decode_kernel<2, KF> : score_decode_kernel<1, KF>;
+  const bool grp = a.group_size > 0;
+  auto kern = a.G > 8 ? (grp ? score_decode_kernel<2, KF, true> : score_decode_kernel<2, KF, false>)
+                      : (grp ? score_decode_kernel<1, KF, true> : score_decode_kernel<1, KF, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, s, a);

@@ -130,7 +130,8 @@ typedef struct {
                                (score descending, lower group id on ties) are kept; sink and
                                local blocks stay whole. k_max * 64 / group_size <= 8192. */
   int32_t k_groups;         /* cap on the kept groups (group_size > 0) */
-  float* group_scores;      /* group_size > 0: device [B, Hkv, nb * 64 / group_size] fp32,
+  float* group_scores;      /* group_size > 0: device [B, Hkv, nb * 64 / group_size] fp32
+                               (16-byte aligned),
                                written by bsa_score_blocks (groups past a sequence: -inf) */
   int32_t* kept_groups;     /* group_size > 0: device [B, Hkv, max_kept] int32, written by
                                bsa_select_top_p: bit k of entry e set when group k of kept
