@@ -34,7 +34,11 @@ namespace bsa {
 namespace {
 
 constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+// Producer warps: one streams whole kept blocks; under two-level routing all of them
+// walk the same quarter sequence and each fills the stages s with s % kProducers equal
+// to its index, so the per-copy issue work is spread over several warps.
+constexpr int kProducers = 4;
+constexpr int kThreads = (kConsumerWarps + kProducers) * 32;
 
 template <int D>
 struct DecodeCfg {
@@ -98,6 +102,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   using Cfg = DecodeCfg<D>;
   using Sm = DecodeSmem<D, NT>;
   constexpr int S = Cfg::kStages;
+  // A producer waits for a ring slot's release by parity, which tells apart only the
+  // phase it waits for and the one before. Its previous own stage (kProducers back)
+  // guaranteed the release of the stage kProducers + S back, so the slot is at most one
+  // phase behind only while kProducers <= S.
+  static_assert(kProducers <= S, "more producers than ring stages");
   constexpr int NH = NT * 8;  // padded heads
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -120,8 +129,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   grid_dependency_wait();   // kept lists come from the selection kernel
 
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------- producer
+  if (warp >= kConsumerWarps) {
+    // ------------------------------------------------------------- producers
+    const int pi = warp - kConsumerWarps;
     // The warp resolves 32 kept entries at a time (block id, then the K and V rows
     // through the page table), one per lane, so the dependent global loads overlap;
     // lane 0 then issues the TMA copies of those blocks back to back.
@@ -135,7 +145,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     constexpr int kW = Sm::kInfoW;
     const bool packed = a.kept_groups != nullptr;
-    uint32_t it = 0;   // stages issued
+    if (!packed && pi != 0) return;   // whole blocks: one producer
+    // the producer that fills stage number k
+    auto owner = [packed](uint32_t k) { return packed ? static_cast<int>(k % kProducers) : 0; };
+    uint32_t it = 0;   // stages issued (by all producers; every producer counts them all)
     bool ok_all = true;
     for (int unit = blockIdx.x; unit < num_units && ok_all; unit += gridDim.x) {
       const int row = unit / a.splits, sp = unit % a.splits;
@@ -205,18 +218,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               // the entry's kept quarters go to the next free slots, one 16-row copy
               // each (issuing whole runs through run-length-dependent branches measured
               // slower); a full stage is handed over once it is known not to be the
-              // unit's last
+              // unit's last. Every producer walks the same sequence; only the owner of a
+              // stage waits for it, fills it and hands it over.
               for (int q4 = 0; q4 < 4 && ok && ok_all; ++q4) {
                 if (!((qm_q >> q4) & 1)) continue;
                 if (open && fill == 4) {
-                  const int s = (it - 1) % S;
-                  sinfo[s * kW + 4] = 0;
-                  mbar_arrive(&full[s]);
+                  if (owner(it - 1) == pi) {
+                    const int s = (it - 1) % S;
+                    sinfo[s * kW + 4] = 0;
+                    mbar_arrive(&full[s]);
+                  }
                   open = false;
                 }
                 if (!open) {
-                  const int s = it % S;
-                  if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
+                  if (owner(it) == pi && !mbar_wait(&empty[it % S], ((it / S) & 1) ^ 1)) {
                     report(a.status, BSA_DEV_TIMEOUT);
                     ok_all = false;
                     break;
@@ -225,16 +240,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                   open = true;
                   fill = 0;
                 }
-                const int s = (it - 1) % S;
-                sinfo[s * kW + fill] = blk_q * kBlock + 16 * q4;
-                unsigned char* st = ring + s * Cfg::kStageBytes + fill * 2048;
-                mbar_expect_tx(&full[s], Cfg::kStageBytes / 4);
+                if (owner(it - 1) == pi) {
+                  const int s = (it - 1) % S;
+                  sinfo[s * kW + fill] = blk_q * kBlock + 16 * q4;
+                  unsigned char* st = ring + s * Cfg::kStageBytes + fill * 2048;
+                  mbar_expect_tx(&full[s], Cfg::kStageBytes / 4);
 #pragma unroll
-                for (int x = 0; x < Cfg::kBoxes; ++x) {
-                  tma_load_2d(st + x * 8192, &tmk16, x * 64, static_cast<int32_t>(rk_q + 16 * q4),
-                              &full[s]);
-                  tma_load_2d(st + Cfg::kTileBytes + x * 8192, &tmv16, x * 64,
-                              static_cast<int32_t>(rv_q + 16 * q4), &full[s]);
+                  for (int x = 0; x < Cfg::kBoxes; ++x) {
+                    tma_load_2d(st + x * 8192, &tmk16, x * 64, static_cast<int32_t>(rk_q + 16 * q4),
+                                &full[s]);
+                    tma_load_2d(st + Cfg::kTileBytes + x * 8192, &tmv16, x * 64,
+                                static_cast<int32_t>(rv_q + 16 * q4), &full[s]);
+                  }
                 }
                 ++fill;
               }
@@ -247,8 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // packed: close the unit's last stage (an empty one when no quarter was kept)
       if (packed && e1 > e0 && ok_all && lane == 0) {
         if (!open) {
-          const int s = it % S;
-          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
+          if (owner(it) == pi && !mbar_wait(&empty[it % S], ((it / S) & 1) ^ 1)) {
             report(a.status, BSA_DEV_TIMEOUT);
             ok_all = false;
           } else {
@@ -257,20 +273,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             fill = 0;
           }
         }
-        if (open) {
+        if (open && owner(it - 1) == pi) {
           const int s = (it - 1) % S;
           for (int w = fill; w < 4; ++w) sinfo[s * kW + w] = -1;
           sinfo[s * kW + 4] = 1;
           mbar_arrive(&full[s]);
         }
+        open = false;
       }
       ok_all = __shfl_sync(0xffffffffu, ok_all ? 1 : 0, 0) != 0;
     }
-    // drain: wait until the consumers released every stage we filled (bounded)
+    // drain: wait until the consumers released every stage this warp filled (bounded)
     if (lane == 0) {
       for (uint32_t k = 0; k < S && k < it; ++k) {
         const uint32_t j = it - 1 - k;
-        mbar_wait(&empty[j % S], (j / S) & 1, 200000000ull);
+        if (owner(j) == pi) mbar_wait(&empty[j % S], (j / S) & 1, 200000000ull);
       }
     }
     return;
