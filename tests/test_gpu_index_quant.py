@@ -191,3 +191,27 @@ def test_quantised_decode_full_size_sampled_rows(fmt):
     xq["k_idx"] = _RowKeys(deq)
     s = parity.compare_decode_rows(w, xq, step, rows)
     print("4-bit full size", s)
+
+
+@pytest.mark.parametrize("fmt", ["fp4", "int4"])
+@pytest.mark.parametrize("gs", [16, 64])
+def test_two_level_routing_on_quantised_cache(fmt, gs):
+    """Two-level routing (HGA, Central mechanism §2) on the 4-bit cache: group scores of
+    the quantised keys, kept groups and attention against the HGA oracle run on the
+    dequantised keys."""
+    w = SMALLQ.with_(p=0.9, k_max=12)
+    x = W.make_decode_inputs(w, "cpu")
+    xd = to_dev(x)
+    prob, qc = quantize_on_device(w, xd, fmt, paged=True)
+    prob.group_size, prob.k_groups = gs, 13
+    step = bsa.DecodeStep(prob)
+    _, K, V = bsa.caches_for(xd)
+    step.run(xd["q"], xd["q_idx"], qc, K, V)
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    _, g, codes, scales = oracle_records(w, x, fmt)
+    xq = dict(x)
+    xq["k_idx"] = torch.from_numpy(iq.dequantize(codes, scales, g, fmt))
+    rows = [(b, gg) for b in range(w.B) for gg in range(w.Hkv)]
+    s = parity.compare_hga_rows(w, xq, step, rows, gs, 13)
+    assert s["rows"] == len(rows)
