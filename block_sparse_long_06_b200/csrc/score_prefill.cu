@@ -133,9 +133,11 @@ __global__ void __launch_bounds__(kWarps * 32) score_prefill_kernel(const ScoreP
       float m = pm[0][threadIdx.x];
 #pragma unroll
       for (int ww = 1; ww < kWarps; ++ww) m = fmaxf(m, pm[ww][threadIdx.x]);
+      // a computed score is >= 0; -inf marks a block that failed validation (its
+      // BSA_DEV_BAD_PAGE is already reported)
       const float sc = a.idx_scale * m;
       out[j0 + threadIdx.x] = sc;
-      if (!isfinite(sc)) report(a.status, BSA_DEV_NONFINITE);
+      if (m != -INFINITY && !isfinite(sc)) report(a.status, BSA_DEV_NONFINITE);
     }
     __syncthreads();
   }
@@ -221,7 +223,7 @@ __global__ void __launch_bounds__(kWarps * 32) score_prefill_g1_kernel(const Sco
       }
       const float sc = bad ? -INFINITY : a.idx_scale * (w * fmaxf(m, 0.f));
       out[j0 + threadIdx.x] = sc;
-      if (!isfinite(sc)) report(a.status, BSA_DEV_NONFINITE);
+      if (!bad && !isfinite(sc)) report(a.status, BSA_DEV_NONFINITE);
     }
     __syncthreads();
   }
