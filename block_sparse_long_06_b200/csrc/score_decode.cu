@@ -101,6 +101,17 @@ BSA_DEVFN uint2 dequant4(uint32_t c16) {
   return make_uint2(w0, w1);
 }
 
+BSA_DEVFN uint32_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+BSA_DEVFN uint32_t lds_u8(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
 // Two FP4 (E2M1) codes in the low byte of x -> f16x2, the low nibble in the low half;
 // every E2M1 value is exact in f16.
 BSA_DEVFN uint32_t e2m1x2_to_f16x2(uint32_t x) {
@@ -320,6 +331,8 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
         if (lane < gpb) gout[lane] = -INFINITY;
       } else {
         const unsigned char* blk = ring + s * kStageBytes + warp * kBlockBytes;
+        const uint32_t blk_s = smem_u32(blk);
+        const bool whole = valid >= kBlock;   // every token of the block exists
         float mx = 0.f;
         // two-level routing: the max of each 16-token group (tile mt) as the bits of a
         // non-negative float (the scores are >= 0, so integer order is float order),
@@ -334,8 +347,8 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
             x0 = *reinterpret_cast<const uint2*>(blk + r0 * 32 + tig * 8);
             x1 = *reinterpret_cast<const uint2*>(blk + r1 * 32 + tig * 8);
           } else if constexpr (KF == 1) {
-            const uint32_t c0 = *reinterpret_cast<const uint16_t*>(blk + r0 * 8 + tig * 2);
-            const uint32_t c1 = *reinterpret_cast<const uint16_t*>(blk + r1 * 8 + tig * 2);
+            const uint32_t c0 = lds_u16(blk_s + r0 * 8 + tig * 2);
+            const uint32_t c1 = lds_u16(blk_s + r1 * 8 + tig * 2);
             x0 = make_uint2(e2m1x2_to_f16x2(c0), e2m1x2_to_f16x2(c0 >> 8));
             x1 = make_uint2(e2m1x2_to_f16x2(c1), e2m1x2_to_f16x2(c1 >> 8));
           } else {
@@ -360,10 +373,13 @@ __global__ void __launch_bounds__(kThreads) score_decode_kernel(const ScoreDecod
           const float send = odd ? vr0 : vr1;
           float keep = odd ? vr1 : vr0;
           keep += __shfl_xor_sync(0xffffffffu, send, 1);
-          keep += __shfl_xor_sync(0xffffffffu, keep, 2);
+          // lanes 2 and 3 of a row group hold heads 4-7 of each 8-head tile: with at most
+          // four heads those are zero-weight padding and the second exchange adds nothing
+          if (NT > 1 || a.G > 4) keep += __shfl_xor_sync(0xffffffffu, keep, 2);
           const int tok = odd ? r1 : r0;
-          if constexpr (KF != 0) keep *= scale_lut[blk[kBlock * 8 + tok] & 0x7Fu];   // token scale
-          if (tok < valid) mx = fmaxf(mx, keep);
+          if constexpr (KF != 0)   // token scale
+            keep *= scale_lut[lds_u8(blk_s + kBlock * 8 + tok) & 0x7Fu];
+          if (whole || tok < valid) mx = fmaxf(mx, keep);
           if constexpr (GRP) gbits[mt] = __reduce_max_sync(0xffffffffu, tok < valid ? __float_as_int(keep) : -1);
         }
         if (GRP && lane == 0) {
