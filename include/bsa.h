@@ -57,7 +57,9 @@ typedef enum {
 /* Bits OR-ed into *dev_status by the kernels. */
 #define BSA_DEV_BAD_PAGE 0x1   /* page id outside [0, num_pages) or block beyond extent: skipped */
 #define BSA_DEV_BAD_KEPT 0x2   /* kept block id outside [0, nb): skipped */
-#define BSA_DEV_NONFINITE 0x4  /* a block score was +-inf or NaN */
+#define BSA_DEV_NONFINITE 0x4  /* a computed block score was +-inf or NaN (a block that
+                                  failed validation is written as -inf and reported as
+                                  BSA_DEV_BAD_PAGE only) */
 #define BSA_DEV_TIMEOUT 0x8    /* a bounded wait inside a kernel gave up; outputs invalid */
 #define BSA_DEV_FP16_RANGE 0x10 /* a value outside the fp16 range: a prefill V value, or an
                                    index query scored against an FP4 index-key cache */
